@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Throughput of the fused weighted GNN aggregation step on B200.
+
+A step is one pass of the whole per-call hot path over one batch of inputs on
+a lowered (fixed) topology: forward Y = A_w X, feature gradient dX = A_w^T dY
+and weight gradient dw_e = dot(X[src_e], dY[dst_e]).  The default workload is
+the R-MAT scale-22 graph (4,194,304 nodes, 67,108,864 edges, H = 128, bf16
+features with fp32 accumulation), whose inputs (X and dY are 1 GiB each) are
+larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs an independent replica (the path has no
+exchange step); the reported value is the sum over ranks of the E*H per step
+divided by the slowest rank's time.  --impl reference times the fp64 CPU
+oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "E·H/s for SpMM fwd, dX and SDDMM dw; achieved HBM GB/s as % of B200 peak"
+UNIT = "E*H/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="rmat22", choices=list(workloads.CONFIGS))
+    p.add_argument("--seed", type=int, default=1)
+    p.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer measurement")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time per sample")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(N, E, H, elem):
+    """Minimal bytes of one call: CSR + order map + weights + input rows read
+    once + output rows written once (dw: both index arrays, dw, X and dY once)."""
+    spmm = 4 * (N + 1) + 4 * E + 4 * E + 4 * E + 2 * N * H * elem
+    dw = 8 * E + 4 * E + 2 * N * H * elem
+    return {"fwd": spmm, "dx": spmm, "dw": dw}
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gnn_sparse_aggregation_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload, kernel_op):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        rec = d.get(workload, {}).get(kernel_op)
+        if rec and rec.get("source_hash") == source_hash():
+            return rec.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile(prefix="clocks", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        self.out.flush()
+        try:
+            rows = [ln.split(",") for ln in open(self.out.name).read().splitlines() if ln.strip()]
+        finally:
+            os.unlink(self.out.name)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The slowest rank's value (every rank calls this at the same point)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_step: int, steps: int, ms: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time."""
+    return world * units_per_step * steps / (ms / 1e3)
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(wl, target_seconds: float):
+    """A bounded sample of the workload for the fp64 CPU oracle: the first S
+    COO edges with their endpoints relabelled compactly (the per-edge work is
+    unchanged; only untouched rows are dropped).  S is chosen so that one
+    fwd + dX + dw pass takes about target_seconds on one core."""
+    import oracle
+    H = wl.H
+    # calibrate on a small prefix
+    def make(S):
+        src = wl.src[:S].cpu().numpy()
+        dst = wl.dst[:S].cpu().numpy()
+        nodes, inv = np.unique(np.concatenate([src, dst]), return_inverse=True)
+        s_loc = inv[:S].astype(np.int32)
+        d_loc = inv[S:].astype(np.int32)
+        idx = torch.from_numpy(nodes).to(wl.X.device).long()
+        X = wl.X[idx].float().cpu().numpy()
+        dY = wl.dY[idx].float().cpu().numpy()
+        w = wl.w[:S].cpu().numpy()
+        return int(nodes.size), s_loc, d_loc, w, X, dY
+
+    def run(sample):
+        n, s, d, w, X, dY = sample
+        t0 = time.perf_counter()
+        oracle.fwd(s, d, n, w, X)
+        oracle.dx(s, d, n, w, dY)
+        oracle.dw(s, d, n, X, dY)
+        return time.perf_counter() - t0
+
+    S = min(wl.E, 1 << 16)
+    t = run(make(S))
+    if S < wl.E:
+        S = int(min(wl.E, max(S, S * target_seconds / max(t, 1e-6))))
+    sample = make(S)
+    return S, sample, run
+
+
+# ----------------------------------------------------------------------------- arms
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = workloads.make(args.workload, seed=args.seed, device=device)
+    S, sample, run = oracle_sample(wl, args.cpu_seconds / max(1, args.steps) * 2)
+    for _ in range(args.warmup):
+        run(sample)
+    t = [run(sample) for _ in range(args.steps)]
+    total = sum(t)
+    value = S * wl.H * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(wl, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"first {S} of {wl.E} COO edges (endpoints relabelled), "
+                                   f"fwd+dX+dw per step, H={wl.H}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, args):
+    return {"workload": f"{wl.name}: N={wl.N}, E={wl.E}, H={wl.H}, "
+                        f"features {str(wl.feature_dtype).replace('torch.', '')}",
+            "N": wl.N, "E": wl.E, "H": wl.H,
+            "feature_dtype": str(wl.feature_dtype).replace("torch.", ""),
+            "weights": "fp32, COO order", "seed": args.seed,
+            "l2": "inputs larger than L2 (X and dY exceed 126 MB), no flush" if wl.N * wl.H * (
+                2 if wl.feature_dtype == torch.bfloat16 else 4) > (126 << 20) else
+                  "inputs smaller than L2: warm-L2 numbers",
+            "step": "ag_spmm_fwd + ag_spmm_dx + ag_sddmm_dw on a lowered graph"}
+
+
+def our_arm(args):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from gnn_sparse_aggregation_b200 import _build
+    if rank == 0 or world == 1:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    import gnn_sparse_aggregation_b200 as agb
+
+    dev = torch.device("cuda", local)
+    wl = workloads.make(args.workload, seed=args.seed, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # lowering (once per topology; reported, not part of the step)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    g = agb.ag_graph_lower(wl.src, wl.dst, wl.N)
+    lower_ms = 1e3 * (time.perf_counter() - t0)
+    st = g.stats
+
+    Y = torch.empty_like(wl.X)
+    dX = torch.empty_like(wl.dY)
+    dw = torch.empty(wl.E, dtype=torch.float32, device=dev)
+    g.scratch(wl.H)
+
+    ops = ("fwd", "dx", "dw")
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        agb.ag_spmm_fwd(g, wl.w, wl.X, Y)
+        if ev is not None:
+            ev[1].record(stream)
+        agb.ag_spmm_dx(g, wl.w, wl.dY, dX)
+        if ev is not None:
+            ev[2].record(stream)
+        agb.ag_sddmm_dw(g, wl.X, wl.dY, dw)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for k in range(K):
+            step(evs[k])
+        end.record(stream)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+    clocks = clk.summary()
+    ms = start.elapsed_time(end)
+    per_op = {op: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)] for i, op in enumerate(ops)}
+    ms = max_over_ranks(ms, dev)
+
+    # end to end from host buffers, copies inside the timed region
+    e2e = None
+    Ke = args.e2e_steps if args.e2e_steps is not None else min(K, 5)
+    if Ke > 0:
+        hw, hX, hdY = (t.cpu().pin_memory() for t in (wl.w, wl.X, wl.dY))
+        hY, hdX = torch.empty_like(hX).pin_memory(), torch.empty_like(hX).pin_memory()
+        hdw = torch.empty_like(hw).pin_memory()
+        staging = torch.empty(agb.ag_step_staging_bytes(g, wl.H, wl.X.dtype), dtype=torch.uint8, device=dev)
+        agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(Ke):
+            agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        elem = hX.element_size()
+        e2e = {"value": whole_job_rate(world, wl.E * wl.H, Ke, e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": hw.numel() * 4 + 2 * hX.numel() * elem,
+               "d2h_bytes_per_step": 2 * hX.numel() * elem + hdw.numel() * 4,
+               "steps": Ke, "ms_per_step": e_ms / Ke}
+        del staging, hw, hX, hdY, hY, hdX, hdw
+
+    hbm, peak_kind = peaks()
+    elem = wl.X.element_size()
+    algo = algorithmic_bytes(wl.N, wl.E, wl.H, elem)
+    avg = {op: sum(v) / len(v) for op, v in per_op.items()}
+    dominant = max(avg, key=avg.get)
+    kernels = {}
+    for op in ops:
+        gbs = algo[op] / (avg[op] / 1e3) / 1e9
+        kernels[op] = {"ms": avg[op], "EH_per_s": wl.E * wl.H / (avg[op] / 1e3),
+                       "algorithmic_bytes": algo[op], "GB_per_s": gbs, "frac_of_peak": gbs / hbm}
+    launches_per_step = (1 + (st["heavy_rows_f"] > 0)) + (1 + (st["heavy_rows_t"] > 0)) + (1 if wl.E else 0)
+    line = {
+        "metric": METRIC,
+        "value": whole_job_rate(world, wl.E * wl.H, K, ms),
+        "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": workload_config(wl, args),
+        "roofline": {"bound": "hbm", "kernel": dominant,
+                     "achieved": algo[dominant] / (avg[dominant] / 1e3) / 1e9,
+                     "peak": hbm, "unit": "GB/s",
+                     "frac": algo[dominant] / (avg[dominant] / 1e3) / 1e9 / hbm,
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": ncu_traffic(args.workload, dominant)},
+        "kernels": kernels,
+        "lowering_ms": lower_ms,
+        "schedule": {k: st[k] for k in ("heavy_rows_f", "chunks_f", "heavy_rows_t", "chunks_t",
+                                        "max_degree_f", "max_degree_t")},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if world > 1:
+        dist.barrier()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        S, sample, run = oracle_sample(wl, args.cpu_seconds)
+        secs = run(sample)
+        line["cpu_baseline"] = {"value": S * wl.H / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"first {S} of {wl.E} COO edges (endpoints relabelled), "
+                                          f"one fwd+dX+dw pass, H={wl.H}, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    g.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+    return our_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,294 @@
+"""Fused weighted GNN aggregation on B200 (sm_100a): Python binding.
+
+This module only marshals torch tensors into the C ABI of ``libaggraph.so``
+(declared in ``include/aggraph.h``); every step of the computation runs in the
+library's CUDA kernels.  There is no CPU fallback: importing this package fails
+if the library has not been built, and every call fails on tensors that are
+not on a CUDA device.
+
+Operations (tinymesh "Weighted aggregation experiment", sections "Decision"
+and "Edge order is explicit"), with A_w[dst_e, src_e] = w_e:
+
+    ag_graph_lower(src, dst, N)  -> Graph   forward CSR + transpose CSR + order maps
+    ag_spmm_fwd(g, w, X)         -> Y  = A_w X
+    ag_spmm_dx(g, w, dY)         -> dX = A_w^T dY
+    ag_sddmm_dw(g, X, dY)        -> dw_e = dot(X[src_e], dY[dst_e])   (COO order)
+    ag_step_host(g, w, X, dY, ...)  the three from host buffers, copies included
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+__all__ = ["AggraphError", "Graph", "ag_graph_lower", "ag_spmm_fwd", "ag_spmm_dx", "ag_sddmm_dw",
+           "ag_step_host", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
+           "declared_symbols", "AG_F32", "AG_BF16"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaggraph.so")
+HEADER_PATH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                           "include", "aggraph.h")
+
+AG_F32, AG_BF16 = 0, 1
+_STATUS = {0: "AG_OK", 1: "AG_ERR_INVALID_ARG", 2: "AG_ERR_SHAPE", 3: "AG_ERR_DTYPE",
+           4: "AG_ERR_DEVICE", 5: "AG_ERR_INDEX_RANGE", 6: "AG_ERR_CUDA", 7: "AG_ERR_WORKSPACE"}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m gnn_sparse_aggregation_b200._build` "
+        "(or __graft_entry__.build()); there is no fallback implementation")
+
+
+class AggraphError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+        self.status_name = _STATUS.get(status, str(status))
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("E", ctypes.c_int64), ("device", ctypes.c_int32),
+                ("chunk_edges", ctypes.c_int32), ("heavy_threshold", ctypes.c_int64),
+                ("max_degree_f", ctypes.c_int64), ("max_degree_t", ctypes.c_int64),
+                ("heavy_rows_f", ctypes.c_int64), ("chunks_f", ctypes.c_int64),
+                ("nonempty_rows_f", ctypes.c_int64), ("heavy_rows_t", ctypes.c_int64),
+                ("chunks_t", ctypes.c_int64), ("nonempty_rows_t", ctypes.c_int64),
+                ("workspace_bytes_used", ctypes.c_size_t)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+_P, _I64, _SZ, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+_PP = ctypes.POINTER(ctypes.c_void_p)
+
+lib = ctypes.CDLL(LIB_PATH)
+lib.ag_graph_workspace_bytes.argtypes = [_I64, _I64]
+lib.ag_graph_workspace_bytes.restype = _SZ
+lib.ag_graph_lower.argtypes = [_P, _P, _I64, _I64, _P, _SZ, _P, _PP]
+lib.ag_graph_arrays.argtypes = [_P] + [_PP] * 6
+lib.ag_graph_get_stats.argtypes = [_P, ctypes.POINTER(Stats)]
+lib.ag_spmm_scratch_bytes.argtypes = [_P, _I64]
+lib.ag_spmm_scratch_bytes.restype = _SZ
+lib.ag_spmm_fwd.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+lib.ag_spmm_dx.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+lib.ag_sddmm_dw.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
+lib.ag_step_staging_bytes.argtypes = [_P, _I64, _I]
+lib.ag_step_staging_bytes.restype = _SZ
+lib.ag_step_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+lib.ag_graph_free.argtypes = [_P]
+lib.ag_graph_free.restype = None
+lib.ag_last_error.restype = ctypes.c_char_p
+lib.ag_status_string.argtypes = [_I]
+lib.ag_status_string.restype = ctypes.c_char_p
+for _name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
+              "ag_sddmm_dw", "ag_step_host", "ag_abi_version"):
+    getattr(lib, _name).restype = _I
+
+
+def declared_symbols(header: str = HEADER_PATH) -> list[str]:
+    """Names of the functions include/aggraph.h declares."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ag_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise AggraphError(rc, lib.ag_last_error().decode(errors="replace"))
+
+
+def _stream(device: torch.device, stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream if hasattr(s, "cuda_stream") else int(s))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return AG_F32
+    if t.dtype == torch.bfloat16:
+        return AG_BF16
+    raise AggraphError(3, f"feature dtype {t.dtype} is not supported (float32 or bfloat16)")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None or t.numel() == 0 else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(name: str, t: torch.Tensor) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise AggraphError(4, f"{name} must be a CUDA tensor (got device {t.device})")
+    if not t.is_contiguous():
+        raise AggraphError(2, f"{name} must be contiguous")
+
+
+def ag_graph_workspace_bytes(N: int, E: int) -> int:
+    return int(lib.ag_graph_workspace_bytes(N, E))
+
+
+class Graph:
+    """A lowered fixed topology (owns its device workspace tensor)."""
+
+    def __init__(self, src: torch.Tensor, dst: torch.Tensor, num_nodes: int, stream=None):
+        for name, t in (("src", src), ("dst", dst)):
+            _need_cuda(name, t)
+            if t.dtype != torch.int32 or t.dim() != 1:
+                raise AggraphError(3 if t.dtype != torch.int32 else 2, f"{name} must be a 1-D int32 tensor")
+        if src.shape != dst.shape:
+            raise AggraphError(2, "src and dst must have the same length")
+        self.device = src.device
+        self.N, self.E = int(num_nodes), int(src.shape[0])
+        nbytes = ag_graph_workspace_bytes(self.N, self.E)
+        if nbytes == 0:
+            raise AggraphError(2, f"unsupported sizes N={self.N}, E={self.E}")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        handle = ctypes.c_void_p()
+        self._h = None
+        _check(lib.ag_graph_lower(_ptr(src), _ptr(dst), self.N, self.E,
+                                  ctypes.c_void_p(self.workspace.data_ptr()), nbytes,
+                                  _stream(self.device, stream), ctypes.byref(handle)))
+        self._h = handle
+        st = Stats()
+        _check(lib.ag_graph_get_stats(self._h, ctypes.byref(st)))
+        self.stats = st.as_dict()
+        self._scratch: dict[int, torch.Tensor] = {}
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise AggraphError(1, "graph is closed")
+        return self._h
+
+    def scratch_bytes(self, H: int) -> int:
+        return int(lib.ag_spmm_scratch_bytes(self.handle, H))
+
+    def scratch(self, H: int) -> torch.Tensor | None:
+        """Device scratch for the split rows at width H (allocated once per H)."""
+        n = self.scratch_bytes(H)
+        if n == 0:
+            return None
+        t = self._scratch.get(H)
+        if t is None:
+            t = torch.empty(n, dtype=torch.uint8, device=self.device)
+            self._scratch[H] = t
+        return t
+
+    def arrays(self) -> dict:
+        """Device int32 views of rowptr_f, col_f, edge_order, rowptr_t, col_t, transpose_order."""
+        ptrs = [ctypes.c_void_p() for _ in range(6)]
+        _check(lib.ag_graph_arrays(self.handle, *[ctypes.byref(p) for p in ptrs]))
+        base = self.workspace.data_ptr()
+        names = ("rowptr_f", "col_f", "edge_order", "rowptr_t", "col_t", "transpose_order")
+        sizes = (self.N + 1, self.E, self.E, self.N + 1, self.E, self.E)
+        out = {}
+        for name, p, n in zip(names, ptrs, sizes):
+            off = (p.value or base) - base
+            out[name] = self.workspace[off:off + 4 * n].view(torch.int32)
+        return out
+
+    def close(self) -> None:
+        if self._h is not None:
+            lib.ag_graph_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # convenience methods
+    def fwd(self, w, X, out=None, stream=None):
+        return ag_spmm_fwd(self, w, X, out, stream)
+
+    def dx(self, w, dY, out=None, stream=None):
+        return ag_spmm_dx(self, w, dY, out, stream)
+
+    def dw(self, X, dY, out=None, stream=None):
+        return ag_sddmm_dw(self, X, dY, out, stream)
+
+
+def ag_graph_lower(src: torch.Tensor, dst: torch.Tensor, N: int, stream=None) -> Graph:
+    return Graph(src, dst, N, stream)
+
+
+def _check_feat(g: Graph, name: str, t: torch.Tensor) -> int:
+    _need_cuda(name, t)
+    if t.dim() != 2 or t.shape[0] != g.N:
+        raise AggraphError(2, f"{name} must be [N={g.N}, H], got {tuple(t.shape)}")
+    return _dtype_code(t)
+
+
+def _check_edge_vec(g: Graph, name: str, t: torch.Tensor) -> None:
+    _need_cuda(name, t)
+    if t.dtype != torch.float32:
+        raise AggraphError(3, f"{name} must be float32")
+    if t.dim() != 1 or t.shape[0] != g.E:
+        raise AggraphError(2, f"{name} must be [E={g.E}], got {tuple(t.shape)}")
+
+
+def _spmm(fn, g: Graph, w, F, out, stream, names):
+    _check_edge_vec(g, "w", w)
+    code = _check_feat(g, names[0], F)
+    H = F.shape[1]
+    if out is None:
+        out = torch.empty_like(F)
+    elif out.shape != F.shape or out.dtype != F.dtype:
+        raise AggraphError(2, f"{names[1]} must match {names[0]} in shape and dtype")
+    else:
+        _need_cuda(names[1], out)
+    scr = g.scratch(H)
+    _check(fn(g.handle, _ptr(w), _ptr(F), _ptr(out), H, code, _ptr(scr),
+              0 if scr is None else scr.numel(), _stream(g.device, stream)))
+    return out
+
+
+def ag_spmm_fwd(g: Graph, w: torch.Tensor, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """Y = A_w X (destination-owned forward CSR)."""
+    return _spmm(lib.ag_spmm_fwd, g, w, X, out, stream, ("X", "Y"))
+
+
+def ag_spmm_dx(g: Graph, w: torch.Tensor, dY: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """dX = A_w^T dY (source-owned transpose CSR)."""
+    return _spmm(lib.ag_spmm_dx, g, w, dY, out, stream, ("dY", "dX"))
+
+
+def ag_sddmm_dw(g: Graph, X: torch.Tensor, dY: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """dw_e = dot(X[src_e], dY[dst_e]) in COO order (float32 [E])."""
+    code = _check_feat(g, "X", X)
+    if _check_feat(g, "dY", dY) != code or dY.shape != X.shape:
+        raise AggraphError(2, "X and dY must have the same shape and dtype")
+    if out is None:
+        out = torch.empty(g.E, dtype=torch.float32, device=g.device)
+    else:
+        _check_edge_vec(g, "dw", out)
+    _check(lib.ag_sddmm_dw(g.handle, _ptr(X), _ptr(dY), _ptr(out), X.shape[1], code,
+                           _stream(g.device, stream)))
+    return out
+
+
+def ag_step_staging_bytes(g: Graph, H: int, dtype: torch.dtype) -> int:
+    code = AG_F32 if dtype == torch.float32 else AG_BF16
+    return int(lib.ag_step_staging_bytes(g.handle, H, code))
+
+
+def ag_step_host(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, Y: torch.Tensor,
+                 dX: torch.Tensor, dw: torch.Tensor, staging: torch.Tensor, stream=None) -> None:
+    """Forward, feature gradient and weight gradient from host buffers.
+
+    w, X, dY are host inputs and Y, dX, dw host outputs (page-locked tensors
+    make the copies asynchronous); staging is a device uint8 tensor of
+    ag_step_staging_bytes(g, H, X.dtype) bytes.  Enqueues on `stream`; the
+    outputs are valid after that stream is synchronized."""
+    for name, t in (("w", w), ("X", X), ("dY", dY), ("Y", Y), ("dX", dX), ("dw", dw)):
+        if t.is_cuda or not t.is_contiguous():
+            raise AggraphError(4, f"{name} must be a contiguous host tensor")
+    code = _dtype_code(X)
+    _need_cuda("staging", staging)
+    _check(lib.ag_step_host(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(Y), _ptr(dX), _ptr(dw),
+                            X.shape[1], code, ctypes.c_void_p(staging.data_ptr()), staging.numel(),
+                            _stream(g.device, stream)))

@@ -1,0 +1,158 @@
+// api.cu -- status handling, pointer checks, workspace layout and handle
+// accessors of libaggraph.  The lowering lives in lower.cu and the per-call
+// kernels in aggregate.cu.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.h"
+
+namespace ag {
+
+static thread_local char g_err[512] = "";
+
+int fail(int status, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int cuda_fail(cudaError_t err, const char *what) {
+    return fail(AG_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(err), cudaGetErrorName(err));
+}
+
+void clear_error() { g_err[0] = '\0'; }
+
+int check_device_ptr(const void *p, int device, const char *name) {
+    cudaPointerAttributes attr;
+    cudaError_t err = cudaPointerGetAttributes(&attr, p);
+    if (err != cudaSuccess) {
+        cudaGetLastError();  // this query's error is not sticky; clear it
+        return fail(AG_ERR_DEVICE, "%s: pointer %p is not known to CUDA (%s)", name, p,
+                    cudaGetErrorString(err));
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+        return fail(AG_ERR_DEVICE, "%s: pointer %p is not device memory", name, p);
+    if (attr.type == cudaMemoryTypeDevice && attr.device != device)
+        return fail(AG_ERR_DEVICE, "%s: pointer %p lives on device %d, graph is on device %d",
+                    name, p, attr.device, device);
+    return AG_OK;
+}
+
+int64_t max_chunks(int64_t E) {
+    // sum over split rows of ceil(deg / C) <= E / C + (number of split rows),
+    // and a split row has more than kHeavyThreshold edges
+    return E / kChunkEdges + E / (kHeavyThreshold + 1) + 1;
+}
+
+static size_t scan_tmp_elems(size_t n) {
+    // one exclusive-scan level per 2048-element tile, recursively, each with a total slot
+    size_t total = 0;
+    while (n > 2048) {
+        n = (n + 2047) / 2048;
+        total += align_up(n + 1, 64);
+    }
+    return total + 64;
+}
+
+bool make_layout(int64_t N, int64_t E, Layout *L) {
+    if (N < 1 || N >= (int64_t(1) << 31) || E < 0 || E >= (int64_t(1) << 31)) return false;
+    const size_t n = size_t(N), e = size_t(E);
+    const size_t m = n > e ? n : e;
+    const size_t tile = 4096;  // radix tile: 256 threads x 16 keys
+    const size_t nblk = (m + tile - 1) / tile;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = off;
+        off += align_up(bytes ? bytes : 1);
+        return at;
+    };
+    for (int d = 0; d < 2; ++d) {
+        L->rowptr[d] = take((n + 1) * 4);
+        L->col[d] = take(e * 4);
+        L->order[d] = take(e * 4);
+        L->rows[d] = take(n * 16);
+        L->chunks[d] = take(size_t(max_chunks(E)) * 16);
+    }
+    // lowering temporaries (unused after ag_graph_lower returns)
+    L->keys_a = take(m * 4);
+    L->vals_a = take(m * 4);
+    L->keys_b = take(m * 4);
+    L->vals_b = take(m * 4);
+    L->hist = take((256 * nblk + 1) * 4);  // +1: the in-place scan writes its total at [n]
+    size_t scan_n = 256 * nblk + 1 > n + 1 ? 256 * nblk + 1 : n + 1;
+    L->scan_tmp = take(scan_tmp_elems(scan_n) * 4);
+    L->aux = take((n + 1) * 4);
+    L->counters = take(64 * 8);
+    L->total = off;
+    return true;
+}
+
+}  // namespace ag
+
+using namespace ag;
+
+extern "C" {
+
+size_t ag_graph_workspace_bytes(int64_t N, int64_t E) {
+    Layout L;
+    if (!make_layout(N, E, &L)) return 0;
+    return L.total;
+}
+
+int ag_graph_arrays(const ag_graph *g, const int32_t **rowptr_f, const int32_t **col_f,
+                    const int32_t **edge_order, const int32_t **rowptr_t, const int32_t **col_t,
+                    const int32_t **transpose_order) {
+    if (!g) return fail(AG_ERR_INVALID_ARG, "ag_graph_arrays: null graph");
+    if (rowptr_f) *rowptr_f = g->dir[0].rowptr;
+    if (col_f) *col_f = g->dir[0].col;
+    if (edge_order) *edge_order = g->dir[0].order;
+    if (rowptr_t) *rowptr_t = g->dir[1].rowptr;
+    if (col_t) *col_t = g->dir[1].col;
+    if (transpose_order) *transpose_order = g->dir[1].order;
+    return AG_OK;
+}
+
+int ag_graph_get_stats(const ag_graph *g, ag_graph_stats *out) {
+    if (!g || !out) return fail(AG_ERR_INVALID_ARG, "ag_graph_get_stats: null argument");
+    memset(out, 0, sizeof *out);
+    out->N = g->N;
+    out->E = g->E;
+    out->device = g->device;
+    out->chunk_edges = kChunkEdges;
+    out->heavy_threshold = kHeavyThreshold;
+    out->max_degree_f = g->dir[0].max_degree;
+    out->max_degree_t = g->dir[1].max_degree;
+    out->heavy_rows_f = g->dir[0].n_heavy;
+    out->chunks_f = g->dir[0].n_chunks;
+    out->nonempty_rows_f = g->dir[0].n_nonempty;
+    out->heavy_rows_t = g->dir[1].n_heavy;
+    out->chunks_t = g->dir[1].n_chunks;
+    out->nonempty_rows_t = g->dir[1].n_nonempty;
+    out->workspace_bytes_used = g->ws_used;
+    return AG_OK;
+}
+
+void ag_graph_free(ag_graph *g) { delete g; }
+
+const char *ag_last_error(void) { return g_err; }
+
+const char *ag_status_string(int status) {
+    switch (status) {
+        case AG_OK: return "AG_OK";
+        case AG_ERR_INVALID_ARG: return "AG_ERR_INVALID_ARG";
+        case AG_ERR_SHAPE: return "AG_ERR_SHAPE";
+        case AG_ERR_DTYPE: return "AG_ERR_DTYPE";
+        case AG_ERR_DEVICE: return "AG_ERR_DEVICE";
+        case AG_ERR_INDEX_RANGE: return "AG_ERR_INDEX_RANGE";
+        case AG_ERR_CUDA: return "AG_ERR_CUDA";
+        case AG_ERR_WORKSPACE: return "AG_ERR_WORKSPACE";
+        default: return "AG_ERR_UNKNOWN";
+    }
+}
+
+int ag_abi_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,216 @@
+/*
+ * aggraph.h -- C ABI of the fused weighted GNN aggregation library
+ * (libaggraph.so, CUDA, sm_100a).
+ *
+ * The operation is the weighted scalar-edge aggregation of the tinymesh page
+ * "Weighted aggregation experiment" (sections "Decision" and "Edge order is
+ * explicit"), which is the fused form of message passing described in the
+ * reading guide "PyTorch Geometric: one abstraction, the whole GNN
+ * literature" (Step 3, "message_and_aggregate is one SpMM"; Step 4, SDDMM):
+ *
+ *   forward          Y  = A_w   X    Y[d, :]  = sum over edges e = (s -> d) of w_e * X[s, :]
+ *   feature grad     dX = A_w^T dY   dX[s, :] = sum over edges e = (s -> d) of w_e * dY[d, :]
+ *   weight grad      dw_e = dot(X[s_e, :], dY[d_e, :])
+ *
+ * A_w[d, s] = w_e, so the forward output is owned by destination rows and the
+ * feature gradient by source rows.  Weights w and their gradient dw stay in
+ * the caller's COO edge order on every call; the library reaches them through
+ * its edge_order / transpose_order maps.  Duplicate (s, d) pairs are separate
+ * edges.  No [E, H] per-edge message tensor is ever formed, and no kernel uses
+ * floating-point atomics, so every output is bitwise reproducible run to run.
+ *
+ * Conventions shared by every entry point
+ *   - Indices are int32; 1 <= N < 2^31 and 0 <= E < 2^31.
+ *   - Feature matrices are dense, row-major, contiguous [N, H] of the given
+ *     dtype (AG_F32: float; AG_BF16: bfloat16 stored as uint16).  w and dw are
+ *     float [E].  Arithmetic is fp32 with fp32 accumulation; bf16 outputs are
+ *     rounded once (round to nearest even) from the fp32 result.
+ *   - All array pointers are DEVICE pointers on the graph's device unless a
+ *     name ends in _host.  The caller owns every buffer; the library never
+ *     allocates device memory.  Pointers must stay valid until the work on
+ *     `stream` has finished.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Per-call functions only enqueue work and return; results are
+ *     ready when the stream reaches that point.
+ *   - Outputs are fully overwritten (never accumulated into).
+ *   - Every int-returning function returns an ag_status; on failure nothing
+ *     is launched and ag_last_error() describes the reason.
+ */
+#ifndef AGGRAPH_H
+#define AGGRAPH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AG_API __attribute__((visibility("default")))
+#else
+#define AG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ag_graph ag_graph; /* opaque lowered topology; fixed once built */
+
+typedef enum ag_dtype {
+    AG_F32 = 0,  /* float32 features */
+    AG_BF16 = 1  /* bfloat16 features (fp32 accumulation) */
+} ag_dtype;
+
+typedef enum ag_status {
+    AG_OK = 0,
+    AG_ERR_INVALID_ARG = 1, /* null handle or pointer, unknown enum value */
+    AG_ERR_SHAPE = 2,       /* N, E or H outside the supported range */
+    AG_ERR_DTYPE = 3,       /* dtype is not AG_F32 or AG_BF16 */
+    AG_ERR_DEVICE = 4,      /* pointer is not device memory of the graph's device */
+    AG_ERR_INDEX_RANGE = 5, /* some src/dst index lies outside [0, N) */
+    AG_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    AG_ERR_WORKSPACE = 7    /* workspace/scratch/staging too small or misaligned */
+} ag_status;
+
+/* Schedule facts of a lowered graph, for inspection and tests. */
+typedef struct ag_graph_stats {
+    int64_t N, E;
+    int32_t device;           /* CUDA ordinal the graph was lowered on */
+    int32_t chunk_edges;      /* heavy rows are split into chunks of this many edges */
+    int64_t heavy_threshold;  /* rows with more in-edges than this are split */
+    int64_t max_degree_f;     /* largest in-degree (forward CSR row length) */
+    int64_t max_degree_t;     /* largest out-degree (transpose CSR row length) */
+    int64_t heavy_rows_f, chunks_f, nonempty_rows_f;
+    int64_t heavy_rows_t, chunks_t, nonempty_rows_t;
+    size_t workspace_bytes_used;
+} ag_graph_stats;
+
+/*
+ * Upper bound on the device workspace ag_graph_lower needs for N nodes and E
+ * edges (256-byte aligned sub-arrays included).  Pure host arithmetic; no
+ * CUDA call.  Returns 0 if N or E is out of range.  The bound is O(N + E):
+ * the two CSRs (2E + 2(N + 1) ints, section "Edge order is explicit"), the
+ * two order maps (2E ints), the row schedules, and sort temporaries.
+ */
+AG_API size_t ag_graph_workspace_bytes(int64_t N, int64_t E);
+
+/*
+ * Connectivity lowering ("Edge order is explicit"; witness in "Exact
+ * witness": edges 0->2, 1->2, 0->1 give edge_order = (2, 0, 1)).
+ *
+ *   src, dst   device int32 [E], the COO edge list (edge e runs src[e] -> dst[e]);
+ *              may be NULL when E == 0.  Read only; they are not retained.
+ *   N, E       node and edge counts.
+ *   workspace  device buffer of at least ag_graph_workspace_bytes(N, E)
+ *              bytes, 256-byte aligned.  The graph lives in it: it must
+ *              outlive the handle and must not be written by the caller.
+ *   stream     stream for the lowering work.  The call synchronizes this
+ *              stream before returning (it reads back validation flags and
+ *              schedule sizes).
+ *   out        receives a new handle (host memory, freed by ag_graph_free).
+ *
+ * Builds, bit-exactly and deterministically:
+ *   rowptr_f[N+1], col_f[E] = src[edge_order], edge_order[E]     (by destination)
+ *   rowptr_t[N+1], col_t[E] = dst[transpose_order], transpose_order[E] (by source)
+ * where each order map sends a CSR position to its COO ordinal, sorted by the
+ * owner key with ties in ascending COO ordinal (a stable sort), plus the
+ * degree-ordered row schedules used by the per-call kernels.
+ *
+ * Errors: AG_ERR_SHAPE for N < 1, E < 0, N or E >= 2^31; AG_ERR_INVALID_ARG
+ * for null out/workspace or null src/dst with E > 0; AG_ERR_WORKSPACE if the
+ * workspace is too small or not 256-byte aligned; AG_ERR_DEVICE if a pointer
+ * is not device memory; AG_ERR_INDEX_RANGE if any index is outside [0, N)
+ * (checked on the device; *out is left unchanged); AG_ERR_CUDA otherwise.
+ */
+AG_API int ag_graph_lower(const int32_t *src, const int32_t *dst, int64_t N, int64_t E,
+                   void *workspace, size_t workspace_bytes, void *stream, ag_graph **out);
+
+/* Device views of the lowered arrays (inside the workspace; any out pointer may be NULL). */
+AG_API int ag_graph_arrays(const ag_graph *g, const int32_t **rowptr_f, const int32_t **col_f,
+                    const int32_t **edge_order, const int32_t **rowptr_t,
+                    const int32_t **col_t, const int32_t **transpose_order);
+
+/* Fills *out with the graph's schedule facts.  AG_ERR_INVALID_ARG on NULL. */
+AG_API int ag_graph_get_stats(const ag_graph *g, ag_graph_stats *out);
+
+/*
+ * Device scratch, in bytes, that ag_spmm_fwd / ag_spmm_dx / ag_step_host need
+ * for feature width H: fp32 partial rows for the chunks of heavy rows
+ * (chunks x H x 4 bytes, the larger of the two directions).  0 when the graph
+ * has no heavy row.  This is O(E / chunk_edges * H), never E x H.
+ */
+AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
+
+/*
+ * Forward aggregation Y = A_w X ("Decision": forward reuses the
+ * destination-owned CSR traversal; reading guide Step 3: the gather / message /
+ * scatter triple is one SpMM when the message is a scalar multiple of the
+ * source row, PyG GraphConv's edge_weight * x_j of section "Reference
+ * contract").
+ *
+ *   w        device float [E], COO order (may be NULL when E == 0)
+ *   X        device [N, H] of dtype
+ *   Y        device [N, H] of dtype, fully written; rows without in-edges are 0
+ *   scratch  device buffer of ag_spmm_scratch_bytes(g, H) bytes (NULL if 0),
+ *            16-byte aligned; its contents are scratch only
+ * Heavy rows are summed in fixed chunk order, so results are bitwise
+ * reproducible.  Errors: AG_ERR_INVALID_ARG, AG_ERR_SHAPE (H < 1 or N*H too
+ * large), AG_ERR_DTYPE, AG_ERR_DEVICE, AG_ERR_WORKSPACE, AG_ERR_CUDA.
+ */
+AG_API int ag_spmm_fwd(const ag_graph *g, const float *w, const void *X, void *Y, int64_t H,
+                int dtype, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
+ * Feature gradient dX = A_w^T dY ("Decision": dX reuses the same CSR
+ * traversal, here over the source-owned transpose CSR and transpose_order).
+ * Arguments and errors as ag_spmm_fwd, with dY in place of X and dX in place
+ * of Y; rows without out-edges are 0.
+ */
+AG_API int ag_spmm_dx(const ag_graph *g, const float *w, const void *dY, void *dX, int64_t H,
+               int dtype, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
+ * Weight gradient dw_e = dot(X[src_e], dY[dst_e]) ("Edge order is explicit";
+ * "Exact witness": one output per edge, reduced over the feature width only;
+ * reading guide Step 4: SDDMM, a dense product evaluated only at the
+ * adjacency's nonzeros).
+ *
+ *   X, dY    device [N, H] of dtype
+ *   dw       device float [E], written in COO order (may be NULL when E == 0)
+ * Every edge's value is computed independently (duplicates get equal values).
+ * Errors as ag_spmm_fwd (no scratch is needed).
+ */
+AG_API int ag_sddmm_dw(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H,
+                int dtype, void *stream);
+
+/*
+ * One whole aggregation step from HOST buffers: copies w, X and dY to the
+ * device staging area, runs forward, feature gradient and weight gradient,
+ * and copies Y, dX and dw back, all enqueued on `stream` in that order.
+ *
+ *   *_host   host buffers (page-locked memory is needed for the copies to be
+ *            asynchronous); w_host/dw_host may be NULL when E == 0
+ *   staging  device buffer of ag_step_staging_bytes(g, H, dtype) bytes,
+ *            256-byte aligned; holds the device copies and the SpMM scratch
+ * The host output buffers are valid once `stream` has been synchronized.
+ */
+AG_API size_t ag_step_staging_bytes(const ag_graph *g, int64_t H, int dtype);
+AG_API int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host,
+                 const void *dY_host, void *Y_host, void *dX_host, float *dw_host,
+                 int64_t H, int dtype, void *staging, size_t staging_bytes, void *stream);
+
+/* Releases the host handle (the caller frees the workspace). NULL is a no-op. */
+AG_API void ag_graph_free(ag_graph *g);
+
+/* Message for the last failure on the calling thread ("" if none). */
+AG_API const char *ag_last_error(void);
+
+/* Static name of a status code. */
+AG_API const char *ag_status_string(int status);
+
+/* Version of this ABI (major * 100 + minor). */
+AG_API int ag_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AGGRAPH_H */

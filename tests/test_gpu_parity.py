@@ -1,0 +1,296 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Element-by-element at every size the oracle finishes in seconds (all of the
+uniform, SBM, R-MAT-16 and 2-hop configurations, the page's witness and its
+edge cases, ragged widths and tails), bit-exact for the lowering, and within
+the stated tolerance for the floating-point outputs.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from tests.gpu_helpers import TOL, TOL_DW, assert_within, check_full, check_lowering, host, lib, run_path
+from tests.golden import load
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def agb():
+    return lib()
+
+
+# ----------------------------------------------------------------------------- witness
+
+def test_witness_through_the_c_abi(agb):
+    g0 = load("witness_3edge.txt")
+    N = g0["N"]
+    src = torch.tensor(g0["src"], dtype=torch.int32, device=DEV)
+    dst = torch.tensor(g0["dst"], dtype=torch.int32, device=DEV)
+    w = torch.tensor(g0["w"], dtype=torch.float32, device=DEV)
+    X = torch.tensor(g0["X"], dtype=torch.float32, device=DEV).reshape(N, 1)
+    dY = torch.tensor(g0["dY"], dtype=torch.float32, device=DEV).reshape(N, 1)
+    g = agb.ag_graph_lower(src, dst, N)
+    arr = g.arrays()
+    for k in ("edge_order", "rowptr_f", "col_f", "transpose_order", "rowptr_t", "col_t"):
+        assert arr[k].cpu().tolist() == g0[k].astype(int).tolist(), k
+    Y = agb.ag_spmm_fwd(g, w, X)
+    dX = agb.ag_spmm_dx(g, w, dY)
+    dw = agb.ag_sddmm_dw(g, X, dY)
+    torch.cuda.synchronize()
+    assert Y[:, 0].cpu().tolist() == g0["Y"].tolist()
+    assert dX[:, 0].cpu().tolist() == g0["dX"].tolist()
+    assert dw.cpu().tolist() == g0["dw"].tolist()
+    # the same through bf16 features (all values are exact in bf16)
+    Yb = agb.ag_spmm_fwd(g, w, X.bfloat16())
+    dXb = agb.ag_spmm_dx(g, w, dY.bfloat16())
+    dwb = agb.ag_sddmm_dw(g, X.bfloat16(), dY.bfloat16())
+    torch.cuda.synchronize()
+    assert Yb[:, 0].float().cpu().tolist() == g0["Y"].tolist()
+    assert dXb[:, 0].float().cpu().tolist() == g0["dX"].tolist()
+    assert dwb.cpu().tolist() == g0["dw"].tolist()
+
+
+# ----------------------------------------------------------------------------- configurations
+
+@pytest.fixture(scope="module", params=["uniform", "sbm", "rmat16", "twohop"])
+def config(request, agb):
+    wl = workloads.make(request.param, seed=1, device=DEV)
+    return wl, agb.ag_graph_lower(wl.src, wl.dst, wl.N)
+
+
+def test_config_lowering_bit_exact(config):
+    wl, g = config
+    check_lowering(g, wl)
+
+
+def test_config_full_parity(config):
+    wl, g = config
+    check_full(g, wl, wl.name)
+
+
+def test_config_bitwise_reproducible(config):
+    wl, g = config
+    a = run_path(g, wl)
+    sc = g.scratch(wl.H)
+    if sc is not None:
+        sc.fill_(0x7f)        # stale scratch contents must not leak into the result
+    b = run_path(g, wl)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8) if x.dtype == torch.bfloat16 else x,
+                           y.view(torch.uint8) if y.dtype == torch.bfloat16 else y)
+
+
+def test_config_no_edge_feature_temporary(config):
+    """No [E, H] carrier: the per-call scratch holds one fp32 row per chunk of
+    a split row, far below E x H (witness section: the largest intermediate is
+    bounded by node state, edge state or row pointers)."""
+    wl, g = config
+    s = g.stats
+    assert g.scratch_bytes(wl.H) == 4 * wl.H * max(s["chunks_f"], s["chunks_t"])
+    assert g.scratch_bytes(wl.H) < wl.E * wl.H * 4 // 16
+    assert g.workspace.numel() < 80 * (wl.N + wl.E) + (1 << 16)
+
+
+def test_rmat16_has_split_rows(config):
+    wl, g = config
+    if wl.name != "rmat16":
+        pytest.skip("split rows are exercised by the R-MAT graph")
+    s = g.stats
+    assert s["heavy_rows_f"] > 0 and s["chunks_f"] > s["heavy_rows_f"]
+    assert s["heavy_rows_t"] > 0 and s["max_degree_f"] > 5000
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+def graph(agb, N, src, dst, H, dtype=torch.float32, seed=5, wdist="normal"):
+    wl = workloads.custom(N, src, dst, H, seed=seed, feature_dtype=dtype, wdist=wdist, device=DEV)
+    return wl, agb.ag_graph_lower(wl.src, wl.dst, wl.N)
+
+
+def skewed_edges(N=3000, E=40000, seed=3):
+    """Random edges plus a hub with 3,000 in-edges and one with 2,500 out-edges
+    (both split), duplicates, self-loops and many empty rows."""
+    rng = np.random.default_rng(seed)
+    src = rng.integers(0, N // 3, E)
+    dst = rng.integers(0, N // 2, E)
+    src = np.concatenate([src, rng.integers(0, N, 3000), np.full(2500, 11)])
+    dst = np.concatenate([dst, np.full(3000, 7), rng.integers(0, N, 2500)])
+    src = np.concatenate([src, [5, 5, 5, 9]])
+    dst = np.concatenate([dst, [6, 6, 6, 9]])
+    perm = rng.permutation(src.size)
+    return N, src[perm].astype(np.int32), dst[perm].astype(np.int32)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("H", [1, 2, 3, 4, 5, 8, 12, 16, 33, 64, 128, 130, 133, 256, 520, 1000, 2056])
+def test_widths_and_split_rows(agb, H, dtype):
+    N, src, dst = skewed_edges()
+    wl, g = graph(agb, N, src, dst, H, dtype)
+    assert g.stats["heavy_rows_f"] >= 1 and g.stats["heavy_rows_t"] >= 1
+    check_full(g, wl, f"H={H} {dtype}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_unaligned_feature_pointers_take_the_narrow_path(agb, dtype):
+    N, src, dst = skewed_edges(N=500, E=6000)
+    H = 64
+    wl, g = graph(agb, N, src, dst, H, dtype)
+    elem = 4 if dtype == torch.float32 else 2
+    off = 1 if dtype == torch.float32 else 1      # one element: breaks 16-byte alignment
+    big = torch.zeros(N * H + off, dtype=dtype, device=DEV)
+    Xu = big[off:].view(N, H)
+    Xu.copy_(wl.X)
+    assert Xu.data_ptr() % 16 == elem * off % 16 != 0
+    Y = g.fwd(wl.w, Xu)
+    ref = g.fwd(wl.w, wl.X)
+    torch.cuda.synchronize()
+    # different vector widths keep the same per-element order of operations
+    assert torch.equal(Y.float(), ref.float())
+
+
+def test_empty_graph_and_one_node(agb):
+    # E = 0: outputs are exact zeros, dw is empty
+    wl, g = graph(agb, 9, [], [], 6)
+    check_lowering(g, wl)
+    Y, dX, dw = run_path(g, wl)
+    assert torch.count_nonzero(Y) == 0 and torch.count_nonzero(dX) == 0 and dw.numel() == 0
+    # N = 1 without and with a self-loop
+    wl, g = graph(agb, 1, [], [], 4)
+    Y, dX, dw = run_path(g, wl)
+    assert torch.count_nonzero(Y) == 0 and dw.numel() == 0
+    wl, g = graph(agb, 1, [0], [0], 4)
+    check_lowering(g, wl)
+    check_full(g, wl, "one node self-loop")
+
+
+def test_isolated_rows_and_duplicates(agb):
+    src = [1, 1, 2, 1, 4, 4]
+    dst = [3, 3, 0, 3, 4, 0]
+    wl, g = graph(agb, 8, src, dst, 5)
+    check_lowering(g, wl)
+    Y, dX, dw = check_full(g, wl, "duplicates")
+    for r in (1, 2, 5, 6, 7):
+        assert torch.count_nonzero(Y[r]) == 0
+    for r in (0, 3, 5, 6, 7):
+        assert torch.count_nonzero(dX[r]) == 0
+    assert dw[0] == dw[1] == dw[3]
+
+
+def test_all_edges_into_one_node(agb):
+    E = 20000
+    rng = np.random.default_rng(1)
+    wl, g = graph(agb, 50, rng.integers(0, 50, E), np.full(E, 42), 32)
+    assert g.stats["max_degree_f"] == E
+    check_lowering(g, wl)
+    check_full(g, wl, "star")
+
+
+def test_many_nodes_few_edges(agb):
+    wl, g = graph(agb, 200_000, [3, 199_999, 17], [199_998, 0, 17], 8)
+    check_lowering(g, wl)
+    check_full(g, wl, "sparse")
+
+
+def test_paired_permutation_keeps_outputs(agb):
+    """Permuting src, dst and w together leaves Y and dX unchanged (within the
+    tolerance: the CSR rows keep the same edges) and permutes dw exactly."""
+    import oracle
+    N, src, dst = skewed_edges(N=800, E=9000)
+    wl, g = graph(agb, N, src, dst, 16)
+    Y, dX, dw = run_path(g, wl)
+    perm = torch.randperm(wl.E, generator=torch.Generator().manual_seed(0)).to(DEV)
+    g2 = agb.ag_graph_lower(wl.src[perm].contiguous(), wl.dst[perm].contiguous(), N)
+    Y2 = g2.fwd(wl.w[perm].contiguous(), wl.X)
+    dX2 = g2.dx(wl.w[perm].contiguous(), wl.dY)
+    dw2 = g2.dw(wl.X, wl.dY)
+    torch.cuda.synchronize()
+    s_, d_, w_ = host(wl.src), host(wl.dst), host(wl.w)
+    _, bY = oracle.fwd(s_, d_, N, w_, host(wl.X), with_bound=True)
+    _, bX = oracle.dx(s_, d_, N, w_, host(wl.dY), with_bound=True)
+    assert_within(Y2, Y.double().cpu().numpy(), bY, 2 * TOL[torch.float32], "permuted fwd")
+    assert_within(dX2, dX.double().cpu().numpy(), bX, 2 * TOL[torch.float32], "permuted dX")
+    assert torch.equal(dw2, dw[perm])       # each edge's dot is computed the same way
+
+
+# ----------------------------------------------------------------------------- API behaviour
+
+def test_non_default_stream(agb):
+    N, src, dst = skewed_edges(N=600, E=7000)
+    wl, g = graph(agb, N, src, dst, 24)
+    ref = run_path(g, wl)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = (g.fwd(wl.w, wl.X, stream=s), g.dx(wl.w, wl.dY, stream=s), g.dw(wl.X, wl.dY, stream=s))
+    s.synchronize()
+    for a, b in zip(ref, out):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_step_from_host_buffers(agb, dtype):
+    N, src, dst = skewed_edges(N=1500, E=20000)
+    wl, g = graph(agb, N, src, dst, 40, dtype)
+    Y, dX, dw = run_path(g, wl)
+    hw, hX, hdY = (t.cpu().pin_memory() for t in (wl.w, wl.X, wl.dY))
+    hY = torch.empty_like(hX).pin_memory()
+    hdX = torch.empty_like(hX).pin_memory()
+    hdw = torch.empty_like(hw).pin_memory()
+    staging = torch.empty(agb.ag_step_staging_bytes(g, wl.H, dtype), dtype=torch.uint8, device=DEV)
+    agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging)
+    torch.cuda.synchronize()
+    assert torch.equal(hY, Y.cpu()) and torch.equal(hdX, dX.cpu()) and torch.equal(hdw, dw.cpu())
+
+
+def test_errors_are_reported_not_launched(agb):
+    N, src, dst = skewed_edges(N=300, E=2000)
+    wl, g = graph(agb, N, src, dst, 8)
+    L = agb.lib
+    Y = torch.empty_like(wl.X)
+    sc = g.scratch(8)
+    sp, sn = (ctypes.c_void_p(sc.data_ptr()), sc.numel()) if sc is not None else (None, 0)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    # host memory where device memory is required
+    hostX = np.zeros((N, 8), np.float32)
+    rc = L.ag_spmm_fwd(g.handle, p(wl.w), hostX.ctypes.data_as(ctypes.c_void_p), p(Y), 8, 0, sp, sn, None)
+    assert rc == 4 and b"device" in L.ag_last_error()
+    pinned = torch.zeros(N, 8).pin_memory()
+    assert L.ag_sddmm_dw(g.handle, p(pinned), p(wl.dY), p(torch.empty(wl.E, device=DEV)), 8, 0, None) == 4
+    # unknown dtype code, bad width
+    assert L.ag_spmm_fwd(g.handle, p(wl.w), p(wl.X), p(Y), 8, 7, sp, sn, None) == 3
+    assert L.ag_spmm_dx(g.handle, p(wl.w), p(wl.dY), p(Y), 0, 0, sp, sn, None) == 2
+    # scratch too small for the split rows
+    N2, s2, d2 = skewed_edges(N=3000, E=1000)
+    wl2, g2 = graph(agb, N2, s2, d2, 8)
+    need = g2.scratch_bytes(8)
+    assert need > 0
+    tiny = torch.empty(16, dtype=torch.uint8, device=DEV)
+    Y2 = torch.empty_like(wl2.X)
+    assert L.ag_spmm_fwd(g2.handle, p(wl2.w), p(wl2.X), p(Y2), 8, 0, p(tiny), 16, None) == 7
+    # index outside [0, N) is caught on the device before anything is built
+    bad_dst = wl.dst.clone()
+    bad_dst[123] = N
+    with pytest.raises(agb.AggraphError) as ei:
+        agb.ag_graph_lower(wl.src, bad_dst, N)
+    assert ei.value.status_name == "AG_ERR_INDEX_RANGE" and "123" in str(ei.value)
+    bad_src = wl.src.clone()
+    bad_src[7] = -1
+    with pytest.raises(agb.AggraphError) as ei:
+        agb.ag_graph_lower(bad_src, wl.dst, N)
+    assert ei.value.status_name == "AG_ERR_INDEX_RANGE"
+    # shape and dtype rejection in the binding
+    with pytest.raises(agb.AggraphError):
+        g.fwd(wl.w[:-1], wl.X)
+    with pytest.raises(agb.AggraphError):
+        g.fwd(wl.w, wl.X[:-1])
+    with pytest.raises(agb.AggraphError):
+        g.fwd(wl.w, wl.X.half())
+    with pytest.raises(agb.AggraphError):
+        g.dw(wl.X, wl.dY.bfloat16())
+    # the context is still healthy after all of the above
+    check_full(g, wl, "after errors")
