@@ -13,6 +13,7 @@ and "Edge order is explicit"), with A_w[dst_e, src_e] = w_e:
     ag_spmm_fwd(g, w, X)         -> Y  = A_w X
     ag_spmm_dx(g, w, dY)         -> dX = A_w^T dY
     ag_sddmm_dw(g, X, dY)        -> dw_e = dot(X[src_e], dY[dst_e])   (COO order)
+    ag_backward(g, w, X, dY)     -> (dX, dw) in one pass over the transpose CSR
     ag_step_host(g, w, X, dY, ...)  the three from host buffers, copies included
 """
 from __future__ import annotations
@@ -23,7 +24,7 @@ import re
 
 import torch
 
-__all__ = ["AggraphError", "Graph", "ag_graph_lower", "ag_spmm_fwd", "ag_spmm_dx", "ag_sddmm_dw",
+__all__ = ["AggraphError", "Graph", "ag_graph_lower", "ag_spmm_fwd", "ag_spmm_dx", "ag_sddmm_dw", "ag_backward",
            "ag_step_host", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
            "declared_symbols", "AG_F32", "AG_BF16"]
 
@@ -50,12 +51,12 @@ class AggraphError(RuntimeError):
 
 class Stats(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("E", ctypes.c_int64), ("device", ctypes.c_int32),
-                ("chunk_edges", ctypes.c_int32), ("heavy_threshold", ctypes.c_int64),
+                ("tile_edges", ctypes.c_int32), ("tiles", ctypes.c_int64),
                 ("max_degree_f", ctypes.c_int64), ("max_degree_t", ctypes.c_int64),
-                ("heavy_rows_f", ctypes.c_int64), ("chunks_f", ctypes.c_int64),
-                ("nonempty_rows_f", ctypes.c_int64), ("heavy_rows_t", ctypes.c_int64),
-                ("chunks_t", ctypes.c_int64), ("nonempty_rows_t", ctypes.c_int64),
-                ("workspace_bytes_used", ctypes.c_size_t)]
+                ("nonempty_rows_f", ctypes.c_int64), ("spanning_rows_f", ctypes.c_int64),
+                ("long_spanning_rows_f", ctypes.c_int64), ("nonempty_rows_t", ctypes.c_int64),
+                ("spanning_rows_t", ctypes.c_int64), ("long_spanning_rows_t", ctypes.c_int64),
+                ("workspace_bytes_used", ctypes.c_size_t), ("dw_locality", ctypes.c_double)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -64,28 +65,34 @@ class Stats(ctypes.Structure):
 _P, _I64, _SZ, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
 _PP = ctypes.POINTER(ctypes.c_void_p)
 
-lib = ctypes.CDLL(LIB_PATH)
-lib.ag_graph_workspace_bytes.argtypes = [_I64, _I64]
-lib.ag_graph_workspace_bytes.restype = _SZ
-lib.ag_graph_lower.argtypes = [_P, _P, _I64, _I64, _P, _SZ, _P, _PP]
-lib.ag_graph_arrays.argtypes = [_P] + [_PP] * 6
-lib.ag_graph_get_stats.argtypes = [_P, ctypes.POINTER(Stats)]
-lib.ag_spmm_scratch_bytes.argtypes = [_P, _I64]
-lib.ag_spmm_scratch_bytes.restype = _SZ
-lib.ag_spmm_fwd.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
-lib.ag_spmm_dx.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
-lib.ag_sddmm_dw.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
-lib.ag_step_staging_bytes.argtypes = [_P, _I64, _I]
-lib.ag_step_staging_bytes.restype = _SZ
-lib.ag_step_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
-lib.ag_graph_free.argtypes = [_P]
-lib.ag_graph_free.restype = None
-lib.ag_last_error.restype = ctypes.c_char_p
-lib.ag_status_string.argtypes = [_I]
-lib.ag_status_string.restype = ctypes.c_char_p
-for _name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
-              "ag_sddmm_dw", "ag_step_host", "ag_abi_version"):
-    getattr(lib, _name).restype = _I
+def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
+    """Declares the C signatures of libaggraph on a loaded library handle."""
+    handle.ag_graph_workspace_bytes.argtypes = [_I64, _I64]
+    handle.ag_graph_workspace_bytes.restype = _SZ
+    handle.ag_graph_lower.argtypes = [_P, _P, _I64, _I64, _P, _SZ, _P, _PP]
+    handle.ag_graph_arrays.argtypes = [_P] + [_PP] * 6
+    handle.ag_graph_get_stats.argtypes = [_P, ctypes.POINTER(Stats)]
+    handle.ag_spmm_scratch_bytes.argtypes = [_P, _I64]
+    handle.ag_spmm_scratch_bytes.restype = _SZ
+    handle.ag_spmm_fwd.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_spmm_dx.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_sddmm_dw.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
+    handle.ag_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_step_staging_bytes.argtypes = [_P, _I64, _I]
+    handle.ag_step_staging_bytes.restype = _SZ
+    handle.ag_step_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_graph_free.argtypes = [_P]
+    handle.ag_graph_free.restype = None
+    handle.ag_last_error.restype = ctypes.c_char_p
+    handle.ag_status_string.argtypes = [_I]
+    handle.ag_status_string.restype = ctypes.c_char_p
+    for name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
+                 "ag_sddmm_dw", "ag_backward", "ag_step_host", "ag_abi_version"):
+        getattr(handle, name).restype = _I
+    return handle
+
+
+lib = _bind(ctypes.CDLL(LIB_PATH))
 
 
 def declared_symbols(header: str = HEADER_PATH) -> list[str]:
@@ -167,7 +174,7 @@ class Graph:
         return int(lib.ag_spmm_scratch_bytes(self.handle, H))
 
     def scratch(self, H: int) -> torch.Tensor | None:
-        """Device scratch for the split rows at width H (allocated once per H)."""
+        """Device scratch for the rows cut by tile boundaries at width H (allocated once per H)."""
         n = self.scratch_bytes(H)
         if n == 0:
             return None
@@ -210,6 +217,9 @@ class Graph:
 
     def dw(self, X, dY, out=None, stream=None):
         return ag_sddmm_dw(self, X, dY, out, stream)
+
+    def backward(self, w, X, dY, dX=None, dw=None, stream=None):
+        return ag_backward(self, w, X, dY, dX, dw, stream)
 
 
 def ag_graph_lower(src: torch.Tensor, dst: torch.Tensor, N: int, stream=None) -> Graph:
@@ -269,6 +279,30 @@ def ag_sddmm_dw(g: Graph, X: torch.Tensor, dY: torch.Tensor, out=None, stream=No
     _check(lib.ag_sddmm_dw(g.handle, _ptr(X), _ptr(dY), _ptr(out), X.shape[1], code,
                            _stream(g.device, stream)))
     return out
+
+
+def ag_backward(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, dX=None, dw=None,
+                stream=None):
+    """(dX, dw) = (A_w^T dY, dot(X[src_e], dY[dst_e])) in one pass over the transpose CSR."""
+    _check_edge_vec(g, "w", w)
+    code = _check_feat(g, "X", X)
+    if _check_feat(g, "dY", dY) != code or dY.shape != X.shape:
+        raise AggraphError(2, "X and dY must have the same shape and dtype")
+    if dX is None:
+        dX = torch.empty_like(dY)
+    elif dX.shape != dY.shape or dX.dtype != dY.dtype:
+        raise AggraphError(2, "dX must match dY in shape and dtype")
+    else:
+        _need_cuda("dX", dX)
+    if dw is None:
+        dw = torch.empty(g.E, dtype=torch.float32, device=g.device)
+    else:
+        _check_edge_vec(g, "dw", dw)
+    H = X.shape[1]
+    scr = g.scratch(H)
+    _check(lib.ag_backward(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(dX), _ptr(dw), H, code, _ptr(scr),
+                           0 if scr is None else scr.numel(), _stream(g.device, stream)))
+    return dX, dw
 
 
 def ag_step_staging_bytes(g: Graph, H: int, dtype: torch.dtype) -> int:

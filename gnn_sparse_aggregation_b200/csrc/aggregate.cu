@@ -20,15 +20,37 @@
 //     group with xor shuffles.
 #include <cuda_bf16.h>
 
+#include <climits>
+
 #include "internal.h"
 
 namespace ag {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kUnroll = 4;  // gathered rows in flight per lane
+// Tunables (compile-time; the defaults are the measured best on B200).
+#ifndef AG_RING_DEPTH
+#define AG_RING_DEPTH 8   // gathered rows in flight per lane group (shared-memory ring)
+#endif
+#ifndef AG_RING_L1
+#define AG_RING_L1 0      // 1: ring copies also allocate in L1 (cp.async.ca), 0: L2 only (.cg)
+#endif
+#ifndef AG_W_STREAM
+#define AG_W_STREAM 1     // 1: weight gathers are loaded evict-first (no reuse to keep in L2)
+#endif
+#ifndef AG_DW_COO
+#define AG_DW_COO 1       // 1: weight gradient walks COO order (coalesced dw, two gathers per edge)
+#endif
+#ifndef AG_MAX_LANES
+#define AG_MAX_LANES 16   // lanes that share one row (fewer lanes: more 16-byte vectors per lane)
+#endif
 
-enum Mode { kSpmm = 1, kSddmm = 2 };
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;     // gathered rows in flight per lane (register path)
+constexpr int kMinBlocks = 4;  // resident CTAs per SM the register path is compiled for
+constexpr int kRingDepth = AG_RING_DEPTH;
+constexpr double kSingleWalkLocality = 0.5;  // see backward()
+
+enum Mode { kSpmm = 1, kSddmm = 2, kBoth = 3 };  // kBoth: feature and weight gradient in one walk
 
 using bf16_t = uint16_t;  // bfloat16 stored as raw bits
 
@@ -39,25 +61,32 @@ __device__ __forceinline__ uint32_t bf16_bits(float f) {
 }
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) { return bf16_bits(a) | (bf16_bits(b) << 16); }
 
-// Read-only gathered rows: non-coherent path, keep in L1/L2.
+// Vector access to VEC consecutive features: gathered rows stay in their
+// storage type ("raw") until they are used, so that several rows in flight
+// cost only their own size in registers.
 template <typename T, int VEC> struct Vec;
 
 template <> struct Vec<float, 4> {
-    static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
-        float4 t = __ldg(reinterpret_cast<const float4 *>(p));
-        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-    }
+    using raw = float4;
+    static __device__ __forceinline__ raw zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+    static __device__ __forceinline__ raw load_raw(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+    static __device__ __forceinline__ void unpack(raw t, float (&v)[4]) { v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w; }
     static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
         __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
     }
 };
 template <> struct Vec<float, 1> {
-    static __device__ __forceinline__ void load(const float *p, float (&v)[1]) { v[0] = __ldg(p); }
+    using raw = float;
+    static __device__ __forceinline__ raw zero() { return 0.f; }
+    static __device__ __forceinline__ raw load_raw(const float *p) { return __ldg(p); }
+    static __device__ __forceinline__ void unpack(raw t, float (&v)[1]) { v[0] = t; }
     static __device__ __forceinline__ void store(float *p, const float (&v)[1]) { __stcs(p, v[0]); }
 };
 template <> struct Vec<bf16_t, 8> {
-    static __device__ __forceinline__ void load(const bf16_t *p, float (&v)[8]) {
-        uint4 t = __ldg(reinterpret_cast<const uint4 *>(p));
+    using raw = uint4;
+    static __device__ __forceinline__ raw zero() { return make_uint4(0u, 0u, 0u, 0u); }
+    static __device__ __forceinline__ raw load_raw(const bf16_t *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
+    static __device__ __forceinline__ void unpack(raw t, float (&v)[8]) {
         v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
         v[4] = bf16_lo(t.z); v[5] = bf16_hi(t.z); v[6] = bf16_lo(t.w); v[7] = bf16_hi(t.w);
     }
@@ -68,22 +97,42 @@ template <> struct Vec<bf16_t, 8> {
     }
 };
 template <> struct Vec<bf16_t, 2> {
-    static __device__ __forceinline__ void load(const bf16_t *p, float (&v)[2]) {
-        uint32_t t = __ldg(reinterpret_cast<const unsigned int *>(p));
-        v[0] = bf16_lo(t); v[1] = bf16_hi(t);
+    using raw = uint32_t;
+    static __device__ __forceinline__ raw zero() { return 0u; }
+    static __device__ __forceinline__ raw load_raw(const bf16_t *p) {
+        return __ldg(reinterpret_cast<const unsigned int *>(p));
     }
+    static __device__ __forceinline__ void unpack(raw t, float (&v)[2]) { v[0] = bf16_lo(t); v[1] = bf16_hi(t); }
     static __device__ __forceinline__ void store(bf16_t *p, const float (&v)[2]) {
         __stcs(reinterpret_cast<unsigned int *>(p), pack_bf16(v[0], v[1]));
     }
 };
 template <> struct Vec<bf16_t, 1> {
-    static __device__ __forceinline__ void load(const bf16_t *p, float (&v)[1]) {
-        v[0] = __uint_as_float(uint32_t(__ldg(reinterpret_cast<const unsigned short *>(p))) << 16);
+    using raw = uint32_t;
+    static __device__ __forceinline__ raw zero() { return 0u; }
+    static __device__ __forceinline__ raw load_raw(const bf16_t *p) {
+        return uint32_t(__ldg(reinterpret_cast<const unsigned short *>(p)));
     }
+    static __device__ __forceinline__ void unpack(raw t, float (&v)[1]) { v[0] = __uint_as_float(t << 16); }
     static __device__ __forceinline__ void store(bf16_t *p, const float (&v)[1]) {
         *reinterpret_cast<unsigned short *>(p) = (unsigned short)bf16_bits(v[0]);
     }
 };
+
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
+    Vec<T, VEC>::unpack(Vec<T, VEC>::load_raw(p), v);
+}
+
+// A weight gathered through edge_order: one 4-byte use per 32-byte sector,
+// with no reuse worth keeping in L2.
+__device__ __forceinline__ float load_w(const float *p) {
+#if AG_W_STREAM
+    return __ldcs(p);
+#else
+    return __ldg(p);
+#endif
+}
 
 // fp32 partial rows (scratch): VEC floats at p, aligned to VEC * 4 bytes.
 template <int VEC>
@@ -115,54 +164,94 @@ __device__ __forceinline__ void add_partial(const float *p, float (&v)[VEC]) {
 }
 
 struct Params {
-    const int4 *rows;     // schedule {row, begin, end, first chunk}
-    const int4 *chunks;   // {begin, end, row, split-row index}
-    const int32_t *col;   // other endpoint per CSR position
-    const int32_t *order; // CSR position -> COO ordinal
-    const float *w;       // COO weights (SpMM)
-    const void *F;        // gathered feature rows
-    const void *R;        // owner feature rows (SDDMM)
-    void *out;            // SpMM output [N, H]
-    float *partial;       // [n_chunks, H] fp32
-    float *dw;            // SDDMM output, COO order
-    int64_t H;
-    int64_t n_chunks;     // items [0, n_chunks) are chunks
-    int64_t row_first;    // items [n_chunks, n_items) are rows[row_first + i]
-    int64_t n_items;
+    const int32_t *col;        // other endpoint per CSR position
+    const int32_t *order;      // CSR position -> COO ordinal
+    const float *w;            // COO weights (SpMM)
+    const int32_t *nz_rows;    // non-empty rows, ascending
+    const int32_t *nz_rowptr;  // their first position, then E
+    const int32_t *tile_nz;    // row (index into nz_rows) holding each tile's first position
+    const int32_t *zero_rows;  // rows without edges (SpMM writes zeros)
+    const void *F;             // gathered feature rows
+    const void *R;             // owner feature rows (SDDMM)
+    void *out;                 // SpMM output [N, H]
+    float *partial;            // [2 * n_tiles, H]: slot 2t = row continued from tile t-1, 2t+1 = row continued in tile t+1
+    float *dw;                 // SDDMM output, COO order
+    int64_t E, H, n_nz;
+    int64_t n_tiles;           // lane groups [0, n_tiles) walk one tile each
+    int64_t n_zero;            // lane groups [n_tiles, n_tiles + n_zero) zero one empty row each
+    int T;                     // positions per tile
     int G, log2G, col_tiles;
 };
 
-// Group of G lanes (G a power of two <= 32) per item.  Each lane owns the
-// column vectors j = tile * G * NV + k * G + lane (k < NV) of the row.
+template <typename T, int VEC, int NV>
+__device__ __forceinline__ void store_row(T *row, int64_t vbase, int G, const bool (&ok)[NV],
+                                          const float (&acc)[NV][VEC]) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+        if (ok[k]) Vec<T, VEC>::store(row + (vbase + int64_t(k) * G) * VEC, acc[k]);
+}
+
+template <int VEC, int NV>
+__device__ __forceinline__ void store_slot(float *slot, int64_t vbase, int G, const bool (&ok)[NV],
+                                           const float (&acc)[NV][VEC]) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+        if (ok[k]) store_partial<VEC>(slot + (vbase + int64_t(k) * G) * VEC, acc[k]);
+}
+
+// One group of G lanes (G a power of two <= 32) walks the T consecutive CSR
+// positions of one tile in order.  Each lane owns the column vectors
+// j = tile * G * NV + k * G + lane (k < NV) of the rows it touches.
+//   kSpmm : out[row] = sum w[order[p]] * F[col[p]] over the row's positions
+//   kSddmm: dw[order[p]] = dot(R[row], F[col[p]])
+// A row that starts and ends inside the tile is written whole; the segment
+// of a row continued from the previous tile goes to partial slot 2t, the
+// segment of a row continued in the next tile to slot 2t+1.
 template <typename T, int VEC, int NV, int MODE, bool ONE_TILE>
-__global__ void __launch_bounds__(kThreads)
-k_aggregate(const Params P) {
+__global__ void __launch_bounds__(kThreads, NV == 1 ? kMinBlocks : (NV == 2 ? 3 : 2))
+k_tiles(const Params P) {
     const int G = P.G;
     const int64_t gid = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> P.log2G;
-    if (gid >= P.n_items) return;
+    if (gid >= P.n_tiles + P.n_zero) return;
     const int gl = threadIdx.x & (G - 1);
     const int lane = threadIdx.x & 31;
     const unsigned gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
-
-    int64_t beg, end, row;
-    float *partial_row = nullptr;
-    if (gid < P.n_chunks) {
-        const int4 c = P.chunks[gid];
-        beg = c.x; end = c.y; row = c.z;
-        if (MODE == kSpmm) partial_row = P.partial + gid * P.H;
-    } else {
-        const int4 r = P.rows[P.row_first + (gid - P.n_chunks)];
-        row = r.x; beg = r.y; end = r.z;
-    }
     const int64_t H = P.H;
     const int64_t HV = H / VEC;
+
+    if (gid >= P.n_tiles) {  // an empty row: zeros
+        T *row = static_cast<T *>(P.out) + int64_t(P.zero_rows[gid - P.n_tiles]) * H;
+        float z[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) z[v] = 0.f;
+        for (int64_t j = gl; j < HV; j += G) Vec<T, VEC>::store(row + j * VEC, z);
+        return;
+    }
+
+    const int64_t p0 = gid * P.T;
+    const int64_t p1 = min(p0 + int64_t(P.T), P.E);
+    const int i0 = P.tile_nz[gid];
     const T *__restrict__ F = static_cast<const T *>(P.F);
+    float *slot_head = P.partial + (2 * gid) * H;
+    float *slot_tail = P.partial + (2 * gid + 1) * H;
 
     for (int tile = 0; tile < (ONE_TILE ? 1 : P.col_tiles); ++tile) {
         const int64_t vbase = int64_t(tile) * G * NV + gl;
         bool colok[NV];
 #pragma unroll
         for (int k = 0; k < NV; ++k) colok[k] = vbase + int64_t(k) * G < HV;
+
+        // current row and a look-ahead window of the next G rows (one per lane)
+        int row = P.nz_rows[i0];
+        int64_t rend = P.nz_rowptr[i0 + 1];
+        bool before = P.nz_rowptr[i0] < p0;
+        int64_t la_base = int64_t(i0) + 1;
+        int la_row = 0, la_end = INT_MAX;
+        if (la_base + gl < P.n_nz) {
+            la_row = P.nz_rows[la_base + gl];
+            la_end = P.nz_rowptr[la_base + gl + 1];
+        }
+        int la_k = 0;
 
         float acc[NV][VEC];
         float own[NV][VEC];
@@ -171,119 +260,654 @@ k_aggregate(const Params P) {
 #pragma unroll
             for (int v = 0; v < VEC; ++v) acc[k][v] = 0.f, own[k][v] = 0.f;
         if (MODE == kSddmm) {
-            const T *Rrow = static_cast<const T *>(P.R) + row * H;
+            const T *Rrow = static_cast<const T *>(P.R) + int64_t(row) * H;
 #pragma unroll
             for (int k = 0; k < NV; ++k)
-                if (colok[k]) Vec<T, VEC>::load(Rrow + (vbase + int64_t(k) * G) * VEC, own[k]);
+                if (colok[k]) load_vec<T, VEC>(Rrow + (vbase + int64_t(k) * G) * VEC, own[k]);
         }
 
-        for (int64_t base = beg; base < end; base += G) {
-            const int64_t p = base + gl;
-            int c = 0, e = 0;
-            float wt = 0.f;
-            if (p < end) {
-                c = __ldcs(P.col + p);
-                e = __ldcs(P.order + p);
-                if (MODE == kSpmm) wt = __ldg(P.w + e);
+        // indices of the first batch
+        int c_cur = 0, e_cur = 0;
+        float w_cur = 0.f;
+        {
+            const int64_t p = p0 + gl;
+            if (p < p1) {
+                c_cur = __ldcs(P.col + p);
+                e_cur = __ldcs(P.order + p);
+                if (MODE == kSpmm) w_cur = load_w(P.w + e_cur);
             }
-            const int n = int(end - base < G ? end - base : G);
+        }
+        for (int64_t base = p0; base < p1; base += G) {
+            // prefetch the next batch's indices while this batch gathers
+            int c_nxt = 0, e_nxt = 0;
+            const int64_t pn = base + G + gl;
+            if (pn < p1) {
+                c_nxt = __ldcs(P.col + pn);
+                e_nxt = __ldcs(P.order + pn);
+            }
+            const int n = int(p1 - base < G ? p1 - base : G);
             for (int j = 0; j < n; j += kUnroll) {
-                float x[kUnroll][NV][VEC];
+                typename Vec<T, VEC>::raw x[kUnroll][NV];
                 float wv[kUnroll];
 #pragma unroll
                 for (int u = 0; u < kUnroll; ++u) {
-                    const int src = __shfl_sync(gmask, c, (j + u) & (G - 1), G);
-                    wv[u] = (MODE == kSpmm) ? __shfl_sync(gmask, wt, (j + u) & (G - 1), G) : 0.f;
+                    const int src = __shfl_sync(gmask, c_cur, (j + u) & (G - 1), G);
+                    wv[u] = (MODE == kSpmm) ? __shfl_sync(gmask, w_cur, (j + u) & (G - 1), G) : 0.f;
                     const T *Frow = F + int64_t(src) * H;
 #pragma unroll
-                    for (int k = 0; k < NV; ++k) {
-                        if (j + u < n && colok[k]) {
-                            Vec<T, VEC>::load(Frow + (vbase + int64_t(k) * G) * VEC, x[u][k]);
-                        } else {
-#pragma unroll
-                            for (int v = 0; v < VEC; ++v) x[u][k][v] = 0.f;
-                        }
-                    }
+                    for (int k = 0; k < NV; ++k)
+                        x[u][k] = (j + u < n && colok[k]) ? Vec<T, VEC>::load_raw(Frow + (vbase + int64_t(k) * G) * VEC)
+                                                          : Vec<T, VEC>::zero();
                 }
-                if (MODE == kSpmm) {
 #pragma unroll
-                    for (int u = 0; u < kUnroll; ++u)
-                        if (j + u < n)
+                for (int u = 0; u < kUnroll; ++u) {
+                    if (j + u >= n) break;
+                    if (base + j + u == rend) {
+                        // the current row ended: write it, move to the next row
+                        if (MODE == kSpmm) {
+                            if (before) store_slot<VEC, NV>(slot_head, vbase, G, colok, acc);
+                            else store_row<T, VEC, NV>(static_cast<T *>(P.out) + int64_t(row) * H, vbase, G,
+                                                       colok, acc);
 #pragma unroll
                             for (int k = 0; k < NV; ++k)
 #pragma unroll
-                                for (int v = 0; v < VEC; ++v) acc[k][v] = fmaf(wv[u], x[u][k][v], acc[k][v]);
-                } else {
-                    float dot[kUnroll];
+                                for (int v = 0; v < VEC; ++v) acc[k][v] = 0.f;
+                        }
+                        before = false;
+                        row = __shfl_sync(gmask, la_row, la_k, G);
+                        rend = __shfl_sync(gmask, la_end, la_k, G);
+                        if (++la_k == G) {
+                            la_base += G;
+                            la_k = 0;
+                            la_row = 0;
+                            la_end = INT_MAX;
+                            if (la_base + gl < P.n_nz) {
+                                la_row = P.nz_rows[la_base + gl];
+                                la_end = P.nz_rowptr[la_base + gl + 1];
+                            }
+                        }
+                        if (MODE == kSddmm) {
+                            const T *Rrow = static_cast<const T *>(P.R) + int64_t(row) * H;
 #pragma unroll
-                    for (int u = 0; u < kUnroll; ++u) {
-                        dot[u] = 0.f;
-#pragma unroll
-                        for (int k = 0; k < NV; ++k)
-#pragma unroll
-                            for (int v = 0; v < VEC; ++v) dot[u] = fmaf(own[k][v], x[u][k][v], dot[u]);
+                            for (int k = 0; k < NV; ++k)
+                                if (colok[k]) load_vec<T, VEC>(Rrow + (vbase + int64_t(k) * G) * VEC, own[k]);
+                        }
                     }
+                    if (MODE == kSpmm) {
 #pragma unroll
-                    for (int u = 0; u < kUnroll; ++u)
-                        for (int o = G >> 1; o > 0; o >>= 1) dot[u] += __shfl_xor_sync(gmask, dot[u], o, G);
-                    if (ONE_TILE) {
+                        for (int k = 0; k < NV; ++k) {
+                            float xf[VEC];
+                            Vec<T, VEC>::unpack(x[u][k], xf);
 #pragma unroll
-                        for (int u = 0; u < kUnroll; ++u)
-                            if (j + u < n && gl == ((j + u) & (G - 1))) P.dw[e] = dot[u];
+                            for (int v = 0; v < VEC; ++v) acc[k][v] = fmaf(wv[u], xf[v], acc[k][v]);
+                        }
                     } else {
-                        // several column tiles: accumulate the partial dots in dw (this
-                        // lane alone owns edge e, so the read-modify-write is race free)
+                        float dot = 0.f;
 #pragma unroll
-                        for (int u = 0; u < kUnroll; ++u)
-                            if (j + u < n && gl == ((j + u) & (G - 1)))
-                                P.dw[e] = tile == 0 ? dot[u] : P.dw[e] + dot[u];
+                        for (int k = 0; k < NV; ++k) {
+                            float xf[VEC];
+                            Vec<T, VEC>::unpack(x[u][k], xf);
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) dot = fmaf(own[k][v], xf[v], dot);
+                        }
+                        for (int o = G >> 1; o > 0; o >>= 1) dot += __shfl_xor_sync(gmask, dot, o, G);
+                        if (gl == ((j + u) & (G - 1))) {
+                            if (ONE_TILE) P.dw[e_cur] = dot;
+                            else P.dw[e_cur] = tile == 0 ? dot : P.dw[e_cur] + dot;
+                        }
                     }
                 }
             }
+            c_cur = c_nxt;
+            e_cur = e_nxt;
+            if (MODE == kSpmm) w_cur = pn < p1 ? load_w(P.w + e_nxt) : 0.f;
         }
         if (MODE == kSpmm) {
-            if (partial_row) {
-#pragma unroll
-                for (int k = 0; k < NV; ++k)
-                    if (colok[k]) store_partial<VEC>(partial_row + (vbase + int64_t(k) * G) * VEC, acc[k]);
-            } else {
-                T *Yrow = static_cast<T *>(P.out) + row * H;
-#pragma unroll
-                for (int k = 0; k < NV; ++k)
-                    if (colok[k]) Vec<T, VEC>::store(Yrow + (vbase + int64_t(k) * G) * VEC, acc[k]);
-            }
+            // the row open at the tile's end
+            if (before) store_slot<VEC, NV>(slot_head, vbase, G, colok, acc);
+            else if (rend > p1) store_slot<VEC, NV>(slot_tail, vbase, G, colok, acc);
+            else store_row<T, VEC, NV>(static_cast<T *>(P.out) + int64_t(row) * H, vbase, G, colok, acc);
         }
     }
 }
 
-// Sum of the partial rows of every split row, in chunk order.
+// ---------------------------------------------------------------------------- shared-memory ring path
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+#if AG_RING_L1
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+#else
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+#endif
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+template <typename T, int VEC>
+__device__ __forceinline__ typename Vec<T, VEC>::raw lds_raw(const uint4 *p) {
+    if constexpr (sizeof(typename Vec<T, VEC>::raw) == 16) {
+        return *reinterpret_cast<const typename Vec<T, VEC>::raw *>(p);
+    } else {
+        return typename Vec<T, VEC>::raw{};
+    }
+}
+
+// Recursive-halving reduce-scatter over the G lanes of a group: on entry lane
+// l holds v[j] = its partial sum for item j (j < G); on exit v[0] of lane l is
+// the total of item l.  G - 1 shuffles for G items.
+template <int G>
+__device__ __forceinline__ float reduce_scatter(float (&v)[G], int gl, unsigned gmask) {
+#pragma unroll
+    for (int s = G / 2; s >= 1; s >>= 1) {
+        const bool upper = gl & s;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+            const float send = upper ? v[i] : v[i + s];
+            const float keep = upper ? v[i + s] : v[i];
+            v[i] = keep + __shfl_xor_sync(gmask, send, s, G);
+        }
+    }
+    return v[0];
+}
+
+// dot product of two raw 16-byte vectors, accumulated in order into c.
+// bf16: fma.rn.f32.bf16 multiplies two bf16 values exactly and adds in fp32
+// with one rounding -- the same result as widening both to fp32 first.
+__device__ __forceinline__ float dot_raw(float4 a, float4 b, float c) {
+    c = fmaf(a.x, b.x, c);
+    c = fmaf(a.y, b.y, c);
+    c = fmaf(a.z, b.z, c);
+    return fmaf(a.w, b.w, c);
+}
+__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\t"
+        "mov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float dot_raw(uint4 a, uint4 b, float c) {
+    c = dot2_bf16(a.x, b.x, c);
+    c = dot2_bf16(a.y, b.y, c);
+    c = dot2_bf16(a.z, b.z, c);
+    return dot2_bf16(a.w, b.w, c);
+}
+
+// Packed fp32 pairs (Blackwell FFMA2): fma.rn.f32x2 rounds each half exactly
+// like fma.rn.f32, so a pair update equals two scalar fmaf calls.
+using f2 = unsigned long long;
+__device__ __forceinline__ f2 pk2(float a, float b) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void up2(f2 r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
+__device__ __forceinline__ f2 ffma2(f2 a, f2 b, f2 c) {
+    f2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// a raw 16-byte vector as fp32 pairs, in element order
+__device__ __forceinline__ void pairs(float4 t, f2 (&p)[2]) { p[0] = pk2(t.x, t.y); p[1] = pk2(t.z, t.w); }
+__device__ __forceinline__ void pairs(uint4 t, f2 (&p)[4]) {
+    p[0] = pk2(bf16_lo(t.x), bf16_hi(t.x));
+    p[1] = pk2(bf16_lo(t.y), bf16_hi(t.y));
+    p[2] = pk2(bf16_lo(t.z), bf16_hi(t.z));
+    p[3] = pk2(bf16_lo(t.w), bf16_hi(t.w));
+}
+
+template <int NV, int VEC>
+__device__ __forceinline__ void unpack_acc(const f2 (&acc)[NV][VEC / 2], float (&o)[NV][VEC]) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i) up2(acc[k][i], o[k][2 * i], o[k][2 * i + 1]);
+}
+
+// Same contract as k_tiles for 16-byte vectors (fp32 x 4, bf16 x 8) and a
+// single column tile, with the lane-group width G and the ring depth D fixed
+// at compile time.  The gathered rows travel global -> shared memory with
+// cp.async: every lane group keeps the rows of the next D positions in flight
+// in its own ring of D slots.  A lane copies, and later reads, only its own
+// 16-byte pieces, so no barrier is needed between copy and read:
+// cp.async.wait_group orders them for the issuing thread.
+//
+// Control flow is uniform across the warp: tile groups fill whole warps
+// (groups [n_tiles, n_tiles_pad) are idle fillers), every group of a warp
+// runs the warp's longest tile length in batches of G positions with its own
+// bounds as predicates, and the shuffles of the common path use the full
+// warp mask.  A batch inside every group's tile runs fully unrolled without
+// bounds checks (slots, shuffle lanes and refill sources are constants).
+// Indices are prefetched two batches ahead and weights one batch ahead.
+// kSddmm reduces the G dot products of an unrolled batch with one
+// reduce-scatter, after which lane j writes the weight gradient of the
+// batch's position j.  kBoth does both on one walk of the transpose CSR: each
+// gathered dY row feeds the feature-gradient row of its source and the dot
+// product of its edge.  Rows are accumulated with packed fp32 pairs.
+template <typename T, int VEC, int NV, int G, int MODE, int D>
+__global__ void __launch_bounds__(kThreads)
+k_tiles_ring(const Params P) {
+    using raw_t = typename Vec<T, VEC>::raw;
+    static_assert(sizeof(raw_t) == 16, "ring path moves 16-byte vectors");
+    static_assert(G >= D && G % D == 0, "ring depth must divide the batch");
+    constexpr unsigned FULL = 0xffffffffu;
+    extern __shared__ uint4 ring[];
+    constexpr int LOG2G = G == 32 ? 5 : G == 16 ? 4 : G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
+    const int64_t gid = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> LOG2G;
+    const int64_t n_tiles_pad = (P.n_tiles + (32 / G) - 1) / (32 / G) * (32 / G);
+    const int gl = threadIdx.x & (G - 1);
+    const int lane = threadIdx.x & 31;
+    const unsigned gmask = (G == 32) ? FULL : (((1u << G) - 1u) << (lane & ~(G - 1)));
+    const int H = int(P.H);
+    const int HV = H / VEC;
+    bool colok[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) colok[k] = gl + k * G < HV;
+
+    if (gid >= n_tiles_pad) {  // warps of empty rows: zeros
+        const int64_t z = gid - n_tiles_pad;
+        if (z >= P.n_zero) return;
+        T *row = static_cast<T *>(P.out) + int64_t(P.zero_rows[z]) * H + gl * VEC;
+        float zero[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) zero[v] = 0.f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (colok[k]) Vec<T, VEC>::store(row + k * G * VEC, zero);
+        return;
+    }
+
+    // this lane's pieces of the ring: slot s, vector k at my[(s * NV + k) * G]
+    const uint4 *my = ring + (threadIdx.x >> LOG2G) * (D * NV * G) + gl;
+    const uint32_t my_s = smem_addr(my);
+    const bool active = gid < P.n_tiles;
+    const int p0 = active ? int(gid) * P.T : 0;
+    const int len = active ? min(P.T, int(P.E) - p0) : 0;
+    const int len_max = __reduce_max_sync(FULL, len);
+    const int len_min = __reduce_min_sync(FULL, len);
+    const T *__restrict__ F = static_cast<const T *>(P.F) + gl * VEC;
+    float *slot_head = P.partial + (2 * gid) * P.H + gl * VEC;
+    float *slot_tail = P.partial + (2 * gid + 1) * P.H + gl * VEC;
+    T *out = static_cast<T *>(P.out) + gl * VEC;
+    const T *R = static_cast<const T *>(P.R) + gl * VEC;
+
+    // the row open at the current position, and the next G rows (one per lane)
+    int row = 0, rend = INT_MAX, la_base = 0;
+    bool before = false;
+    if (active) {
+        const int i0 = P.tile_nz[gid];
+        row = P.nz_rows[i0];
+        rend = P.nz_rowptr[i0 + 1];
+        before = P.nz_rowptr[i0] < p0;
+        la_base = i0 + 1;
+    }
+    int la_row = 0, la_end = INT_MAX;
+    if (active && la_base + gl < P.n_nz) {
+        la_row = P.nz_rows[la_base + gl];
+        la_end = P.nz_rowptr[la_base + gl + 1];
+    }
+    int la_k = 0;
+
+    // indices: batch b (cur), b + 1 (nxt), b + 2 (nn); weights of b and b + 1
+    int c_cur = 0, e_cur = 0, c_nxt = 0, e_nxt = 0, c_nn = 0, e_nn = 0;
+    float w_cur = 0.f, w_nxt = 0.f;
+    if (gl < len) { c_cur = __ldcs(P.col + p0 + gl); e_cur = __ldcs(P.order + p0 + gl); }
+    if (G + gl < len) { c_nxt = __ldcs(P.col + p0 + G + gl); e_nxt = __ldcs(P.order + p0 + G + gl); }
+    if ((MODE & kSpmm) && gl < len) w_cur = load_w(P.w + e_cur);
+
+    auto issue = [&](int slot, int src) {
+        const T *Frow = F + int64_t(src) * H;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (colok[k]) cp_async16(my_s + uint32_t((slot * NV + k) * G * 16), Frow + k * G * VEC);
+    };
+#pragma unroll
+    for (int s = 0; s < D; ++s) {
+        const int src = __shfl_sync(FULL, c_cur, s, G);
+        if (s < len) issue(s, src);
+        cp_async_commit();
+    }
+
+    f2 acc[NV][VEC / 2];
+    raw_t own[NV], own_next[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        own[k] = own_next[k] = Vec<T, VEC>::zero();
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i) acc[k][i] = 0ull;
+    }
+    if ((MODE & kSddmm) && active) {
+        const T *Rrow = R + int64_t(row) * H;
+        const T *Rnext = R + int64_t(__shfl_sync(gmask, la_row, 0, G)) * H;
+        const bool has_next = la_base < P.n_nz;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (colok[k]) {
+                own[k] = Vec<T, VEC>::load_raw(Rrow + k * G * VEC);
+                if (has_next) own_next[k] = Vec<T, VEC>::load_raw(Rnext + k * G * VEC);
+            }
+    }
+
+    auto write_open_row = [&](float *slot) {
+        float o[NV][VEC];
+        unpack_acc<NV, VEC>(acc, o);
+        if (slot) store_slot<VEC, NV>(slot, 0, G, colok, o);
+        else store_row<T, VEC, NV>(out + int64_t(row) * H, 0, G, colok, o);
+    };
+    // the current row ended at the current position: write it, open the next
+    // (runs only in the lane groups whose row ended: group-mask shuffles)
+    auto next_row = [&]() {
+        if ((MODE & kSpmm)) {
+            write_open_row(before ? slot_head : nullptr);
+#pragma unroll
+            for (int q = 0; q < NV; ++q)
+#pragma unroll
+                for (int i = 0; i < VEC / 2; ++i) acc[q][i] = 0ull;
+        }
+        before = false;
+        row = __shfl_sync(gmask, la_row, la_k, G);
+        rend = __shfl_sync(gmask, la_end, la_k, G);
+        if (++la_k == G) {
+            la_base += G;
+            la_k = 0;
+            la_row = 0;
+            la_end = INT_MAX;
+            if (la_base + gl < P.n_nz) {
+                la_row = P.nz_rows[la_base + gl];
+                la_end = P.nz_rowptr[la_base + gl + 1];
+            }
+        }
+        if ((MODE & kSddmm)) {
+            const T *Rnext = R + int64_t(__shfl_sync(gmask, la_row, la_k, G)) * H;
+            const bool has_next = la_base + la_k < P.n_nz;
+#pragma unroll
+            for (int q = 0; q < NV; ++q) {
+                own[q] = own_next[q];
+                if (colok[q] && has_next) own_next[q] = Vec<T, VEC>::load_raw(Rnext + q * G * VEC);
+            }
+        }
+    };
+    // position p0 + base + j (valid: inside this group's tile); returns this
+    // lane's part of the dot (kSddmm)
+    auto consume = [&](int base, int j, bool valid) -> float {
+        cp_async_wait<D - 1>();
+        const float wk = ((MODE & kSpmm)) ? __shfl_sync(FULL, w_cur, j, G) : 0.f;
+        float d = 0.f;
+        if (valid) {
+            raw_t x[NV];
+#pragma unroll
+            for (int q = 0; q < NV; ++q) x[q] = *reinterpret_cast<const raw_t *>(my + ((j % D) * NV + q) * G);
+            if (p0 + base + j == rend) next_row();
+            // slots of out-of-range column vectors were never written: skip them
+            if ((MODE & kSpmm)) {
+                const f2 w2 = pk2(wk, wk);
+#pragma unroll
+                for (int q = 0; q < NV; ++q) {
+                    if (!colok[q]) continue;
+                    f2 xp[VEC / 2];
+                    pairs(x[q], xp);
+#pragma unroll
+                    for (int i = 0; i < VEC / 2; ++i) acc[q][i] = ffma2(w2, xp[i], acc[q][i]);
+                }
+            }
+            if ((MODE & kSddmm)) {
+#pragma unroll
+                for (int q = 0; q < NV; ++q)
+                    if (colok[q]) d = dot_raw(own[q], x[q], d);
+            }
+        }
+        return d;
+    };
+    // refill slot j % D with position base + j + D (this batch or the next)
+    auto refill = [&](int base, int j, bool check) {
+        const int src = (j + D < G) ? __shfl_sync(FULL, c_cur, (j + D) & (G - 1), G)
+                                    : __shfl_sync(FULL, c_nxt, (j + D) & (G - 1), G);
+        if (!check || base + j + D < len) issue(j % D, src);
+        cp_async_commit();
+    };
+
+    for (int base = 0; base < len_max; base += G) {
+        if (base > 0) {
+            c_cur = c_nxt; e_cur = e_nxt; w_cur = w_nxt;
+            c_nxt = c_nn; e_nxt = e_nn;
+        }
+        // weights of the next batch, indices of the one after
+        if ((MODE & kSpmm)) w_nxt = (base + G + gl < len) ? load_w(P.w + e_nxt) : 0.f;
+        c_nn = 0;
+        e_nn = 0;
+        if (base + 2 * G + gl < len) {
+            c_nn = __ldcs(P.col + p0 + base + 2 * G + gl);
+            e_nn = __ldcs(P.order + p0 + base + 2 * G + gl);
+        }
+        if (base + G + D <= len_min) {
+            float dots[G];
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                dots[j] = consume(base, j, true);
+                refill(base, j, false);
+            }
+            if ((MODE & kSddmm)) P.dw[e_cur] = reduce_scatter<G>(dots, gl, FULL);
+        } else {
+#pragma unroll 1
+            for (int j = 0; j < G; ++j) {
+                float d = consume(base, j, base + j < len);
+                if ((MODE & kSddmm)) {
+#pragma unroll
+                    for (int o = G / 2; o > 0; o >>= 1) d += __shfl_xor_sync(FULL, d, o, G);
+                    if (gl == j && base + j < len) P.dw[e_cur] = d;
+                }
+                refill(base, j, true);
+            }
+        }
+    }
+    if ((MODE & kSpmm) && active) {
+        if (before) write_open_row(slot_head);
+        else if (rend > p0 + len) write_open_row(slot_tail);
+        else write_open_row(nullptr);
+    }
+    cp_async_wait<0>();
+}
+
+// Weight gradient in COO order: lane group per tile of T consecutive COO
+// ordinals; both endpoint rows (X[src_e], dY[dst_e]) travel through the
+// shared-memory ring, and after the batch reduce-scatter lane j writes dw of
+// the batch's ordinal j, so the dw stores are coalesced.  The per-lane
+// partial dots and the reduction tree are those of the CSR walk, so both
+// walks give bitwise identical dw.
+template <typename T, int VEC, int NV, int G, int D>
+__global__ void __launch_bounds__(kThreads)
+k_dw_coo(const int32_t *__restrict__ src, const int32_t *__restrict__ dst, const void *Xv, const void *dYv,
+         float *__restrict__ dw, int E, int H, int T_tile, int64_t n_tiles) {
+    using raw_t = typename Vec<T, VEC>::raw;
+    static_assert(sizeof(raw_t) == 16 && G >= D && G % D == 0, "ring layout");
+    constexpr unsigned FULL = 0xffffffffu;
+    extern __shared__ uint4 ring[];
+    constexpr int LOG2G = G == 32 ? 5 : G == 16 ? 4 : G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
+    const int64_t gid = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> LOG2G;
+    const int gl = threadIdx.x & (G - 1);
+    const int HV = H / VEC;
+    bool colok[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) colok[k] = gl + k * G < HV;
+    // slot s: X piece k at my[((2s) * NV + k) * G], dY piece k at my[((2s + 1) * NV + k) * G]
+    const uint4 *my = ring + (threadIdx.x >> LOG2G) * (2 * D * NV * G) + gl;
+    const uint32_t my_s = smem_addr(my);
+    const bool active = gid < n_tiles;
+    const int p0 = active ? int(gid) * T_tile : 0;
+    const int len = active ? min(T_tile, E - p0) : 0;
+    const int len_max = __reduce_max_sync(FULL, len);
+    const int len_min = __reduce_min_sync(FULL, len);
+    const T *X = static_cast<const T *>(Xv) + gl * VEC;
+    const T *dY = static_cast<const T *>(dYv) + gl * VEC;
+
+    int s_cur = 0, d_cur = 0, s_nxt = 0, d_nxt = 0, s_nn = 0, d_nn = 0;
+    if (gl < len) { s_cur = __ldcs(src + p0 + gl); d_cur = __ldcs(dst + p0 + gl); }
+    if (G + gl < len) { s_nxt = __ldcs(src + p0 + G + gl); d_nxt = __ldcs(dst + p0 + G + gl); }
+
+    auto issue = [&](int slot, int sv, int dv) {
+        const T *xr = X + int64_t(sv) * H;
+        const T *yr = dY + int64_t(dv) * H;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (colok[k]) {
+                cp_async16(my_s + uint32_t(((2 * slot) * NV + k) * G * 16), xr + k * G * VEC);
+                cp_async16(my_s + uint32_t(((2 * slot + 1) * NV + k) * G * 16), yr + k * G * VEC);
+            }
+    };
+#pragma unroll
+    for (int q = 0; q < D; ++q) {
+        const int sv = __shfl_sync(FULL, s_cur, q, G), dv = __shfl_sync(FULL, d_cur, q, G);
+        if (q < len) issue(q, sv, dv);
+        cp_async_commit();
+    }
+    auto consume = [&](int j, bool valid) -> float {
+        cp_async_wait<D - 1>();
+        float d = 0.f;
+        if (valid) {
+#pragma unroll
+            for (int q = 0; q < NV; ++q)
+                if (colok[q]) {
+                    const raw_t a = *reinterpret_cast<const raw_t *>(my + ((2 * (j % D)) * NV + q) * G);
+                    const raw_t b = *reinterpret_cast<const raw_t *>(my + ((2 * (j % D) + 1) * NV + q) * G);
+                    d = dot_raw(a, b, d);
+                }
+        }
+        return d;
+    };
+    auto refill = [&](int base, int j, bool check) {
+        const int lanej = (j + D) & (G - 1);
+        const int sv = (j + D < G) ? __shfl_sync(FULL, s_cur, lanej, G) : __shfl_sync(FULL, s_nxt, lanej, G);
+        const int dv = (j + D < G) ? __shfl_sync(FULL, d_cur, lanej, G) : __shfl_sync(FULL, d_nxt, lanej, G);
+        if (!check || base + j + D < len) issue(j % D, sv, dv);
+        cp_async_commit();
+    };
+    for (int base = 0; base < len_max; base += G) {
+        if (base > 0) {
+            s_cur = s_nxt; d_cur = d_nxt;
+            s_nxt = s_nn; d_nxt = d_nn;
+        }
+        s_nn = 0;
+        d_nn = 0;
+        if (base + 2 * G + gl < len) {
+            s_nn = __ldcs(src + p0 + base + 2 * G + gl);
+            d_nn = __ldcs(dst + p0 + base + 2 * G + gl);
+        }
+        if (base + G + D <= len_min) {
+            float dots[G];
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                dots[j] = consume(j, true);
+                refill(base, j, false);
+            }
+            __stcs(dw + p0 + base + gl, reduce_scatter<G>(dots, gl, FULL));
+        } else {
+#pragma unroll 1
+            for (int j = 0; j < G; ++j) {
+                float d = consume(j, base + j < len);
+#pragma unroll
+                for (int o = G / 2; o > 0; o >>= 1) d += __shfl_xor_sync(FULL, d, o, G);
+                if (gl == j && base + j < len) dw[p0 + base + j] = d;
+                refill(base, j, true);
+            }
+        }
+    }
+    cp_async_wait<0>();
+}
+
+// Rows cut by tile boundaries: out[row] = slot(2 * first + 1) + sum over the
+// following tiles t of slot(2t), in tile order.  Blocks [0, n_long) take one
+// long span each with the whole CTA: lane group q < kStripes adds the tiles
+// t = first + 1 + q, first + 1 + q + kStripes, ... in order, and group 0 then
+// adds the stripes in order.  The stripe count is fixed, so the result does
+// not depend on the lane-group width.  The remaining blocks take one span per
+// lane group, added sequentially.
+constexpr int kStripes = 8;
+
 template <typename T, int VEC, int NV>
 __global__ void __launch_bounds__(kThreads)
-k_finish(const int4 *__restrict__ rows, int64_t n_heavy, const float *__restrict__ partial, void *out,
-         int64_t H, int G, int log2G, int col_tiles) {
-    const int64_t h = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> log2G;
-    if (h >= n_heavy) return;
+k_fixup(const int4 *__restrict__ spans, int64_t n_long, int64_t n_span, const float *__restrict__ partial,
+        void *out, int64_t H, int G, int log2G, int col_tiles) {
+    __shared__ float red[kStripes * 32 * NV * VEC];
     const int gl = threadIdx.x & (G - 1);
-    const int4 r = rows[h];
-    const int nch = (r.z - r.y + kChunkEdges - 1) / kChunkEdges;
+    const int gi = threadIdx.x >> log2G;
+    const int ng = kThreads >> log2G;
     const int64_t HV = H / VEC;
+    if (blockIdx.x < n_long) {
+        const int4 sp = spans[blockIdx.x];
+        for (int tile = 0; tile < col_tiles; ++tile) {
+            const int64_t vbase = int64_t(tile) * G * NV + gl;
+            bool ok[NV];
+#pragma unroll
+            for (int k = 0; k < NV; ++k) ok[k] = vbase + int64_t(k) * G < HV;
+            float acc[NV][VEC];
+#pragma unroll
+            for (int k = 0; k < NV; ++k)
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) acc[k][v] = 0.f;
+            if (gi < kStripes) {
+                if (gi == 0) {
+                    const float *s0 = partial + (2 * int64_t(sp.y) + 1) * H;
+#pragma unroll
+                    for (int k = 0; k < NV; ++k)
+                        if (ok[k]) add_partial<VEC>(s0 + (vbase + int64_t(k) * G) * VEC, acc[k]);
+                }
+                for (int64_t t = sp.y + 1 + gi; t <= sp.z; t += kStripes) {
+                    const float *s1 = partial + (2 * t) * H;
+#pragma unroll
+                    for (int k = 0; k < NV; ++k)
+                        if (ok[k]) add_partial<VEC>(s1 + (vbase + int64_t(k) * G) * VEC, acc[k]);
+                }
+#pragma unroll
+                for (int k = 0; k < NV; ++k)
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) red[(gi * G * NV + k * G + gl) * VEC + v] = acc[k][v];
+            }
+            __syncthreads();
+            if (gi == 0) {
+                for (int q = 1; q < kStripes; ++q)
+#pragma unroll
+                    for (int k = 0; k < NV; ++k)
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) acc[k][v] += red[(q * G * NV + k * G + gl) * VEC + v];
+                T *row = static_cast<T *>(out) + int64_t(sp.x) * H;
+                store_row<T, VEC, NV>(row, vbase, G, ok, acc);
+            }
+            __syncthreads();
+        }
+        return;
+    }
+    const int64_t s = n_long + (int64_t(blockIdx.x) - n_long) * ng + gi;
+    if (s >= n_span) return;
+    const int4 sp = spans[s];
     for (int tile = 0; tile < col_tiles; ++tile) {
         const int64_t vbase = int64_t(tile) * G * NV + gl;
+        bool ok[NV];
+#pragma unroll
+        for (int k = 0; k < NV; ++k) ok[k] = vbase + int64_t(k) * G < HV;
         float acc[NV][VEC];
 #pragma unroll
         for (int k = 0; k < NV; ++k)
 #pragma unroll
             for (int v = 0; v < VEC; ++v) acc[k][v] = 0.f;
-        for (int c = 0; c < nch; ++c) {
-            const float *prow = partial + (int64_t(r.w) + c) * H;
-#pragma unroll
-            for (int k = 0; k < NV; ++k)
-                if (vbase + int64_t(k) * G < HV) add_partial<VEC>(prow + (vbase + int64_t(k) * G) * VEC, acc[k]);
-        }
-        T *Yrow = static_cast<T *>(out) + int64_t(r.x) * H;
+        const float *s0 = partial + (2 * int64_t(sp.y) + 1) * H;
 #pragma unroll
         for (int k = 0; k < NV; ++k)
-            if (vbase + int64_t(k) * G < HV) Vec<T, VEC>::store(Yrow + (vbase + int64_t(k) * G) * VEC, acc[k]);
+            if (ok[k]) add_partial<VEC>(s0 + (vbase + int64_t(k) * G) * VEC, acc[k]);
+        for (int64_t t = sp.y + 1; t <= sp.z; ++t) {
+            const float *s1 = partial + (2 * t) * H;
+#pragma unroll
+            for (int k = 0; k < NV; ++k)
+                if (ok[k]) add_partial<VEC>(s1 + (vbase + int64_t(k) * G) * VEC, acc[k]);
+        }
+        store_row<T, VEC, NV>(static_cast<T *>(out) + int64_t(sp.x) * H, vbase, G, ok, acc);
     }
 }
 
@@ -321,7 +945,7 @@ Shape pick_shape(int64_t H, int dtype, const void *a, const void *b, const void 
     s.vec = vec;
     const int64_t HV = H / vec;
     int G = 1;
-    while (G < 32 && G < HV) G <<= 1;
+    while (G < AG_MAX_LANES && G < HV) G <<= 1;
     s.G = G;
     s.log2G = log2i(G);
     const int64_t per_lane = (HV + G - 1) / G;
@@ -330,21 +954,53 @@ Shape pick_shape(int64_t H, int dtype, const void *a, const void *b, const void 
     return s;
 }
 
+template <typename T, int VEC, int NV, int G, int MODE>
+void launch_ring(const Params &P, cudaStream_t st) {
+    constexpr int D = kRingDepth < G ? kRingDepth : G;
+    // tile groups padded to whole warps, then the empty-row groups
+    const int64_t per_warp = 32 / G;
+    const int64_t groups = (P.n_tiles + per_warp - 1) / per_warp * per_warp + P.n_zero;
+    const unsigned grid = unsigned((groups + kThreads / G - 1) / (kThreads / G));
+    // ring: D slots x NV vectors x 16 bytes for every lane of the block
+    const size_t smem = size_t(kThreads) * D * NV * 16;
+    static bool configured = false;  // per instantiation: the attribute belongs to the function
+    if (!configured) {
+        cudaFuncSetAttribute(k_tiles_ring<T, VEC, NV, G, MODE, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+        configured = true;
+    }
+    k_tiles_ring<T, VEC, NV, G, MODE, D><<<grid, kThreads, smem, st>>>(P);
+}
+
 template <typename T, int VEC, int NV, int MODE>
 void launch_main(const Params &P, const Shape &s, cudaStream_t st) {
     const int64_t groups_per_block = kThreads / s.G;
-    const unsigned grid = unsigned((P.n_items + groups_per_block - 1) / groups_per_block);
-    if (s.col_tiles == 1) k_aggregate<T, VEC, NV, MODE, true><<<grid, kThreads, 0, st>>>(P);
-    else k_aggregate<T, VEC, NV, MODE, false><<<grid, kThreads, 0, st>>>(P);
+    const int64_t groups = P.n_tiles + P.n_zero;
+    const unsigned grid = unsigned((groups + groups_per_block - 1) / groups_per_block);
+    if constexpr (sizeof(typename Vec<T, VEC>::raw) == 16 && NV <= 2) {
+        if (s.col_tiles == 1 && s.G >= 4) {
+            switch (s.G) {
+                case 4: launch_ring<T, VEC, NV, 4, MODE>(P, st); return;
+                case 8: launch_ring<T, VEC, NV, 8, MODE>(P, st); return;
+                case 16: launch_ring<T, VEC, NV, 16, MODE>(P, st); return;
+                default: launch_ring<T, VEC, NV, 32, MODE>(P, st); return;
+            }
+        }
+    }
+    if constexpr (MODE != kBoth) {
+        if (s.col_tiles == 1) k_tiles<T, VEC, NV, MODE, true><<<grid, kThreads, 0, st>>>(P);
+        else k_tiles<T, VEC, NV, MODE, false><<<grid, kThreads, 0, st>>>(P);
+    }
 }
 
 template <typename T, int VEC, int NV>
-void launch_finish(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s,
-                   cudaStream_t st) {
+void launch_fixup(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s,
+                  cudaStream_t st) {
     const int64_t groups_per_block = kThreads / s.G;
-    const unsigned grid = unsigned((D.n_heavy + groups_per_block - 1) / groups_per_block);
-    k_finish<T, VEC, NV><<<grid, kThreads, 0, st>>>(D.rows, D.n_heavy, partial, out, H, s.G, s.log2G,
-                                                    s.col_tiles);
+    const int64_t short_spans = D.n_span - D.n_span_long;
+    const unsigned grid = unsigned(D.n_span_long + (short_spans + groups_per_block - 1) / groups_per_block);
+    k_fixup<T, VEC, NV><<<grid, kThreads, 0, st>>>(D.spans, D.n_span_long, D.n_span, partial, out, H, s.G,
+                                                   s.log2G, s.col_tiles);
 }
 
 template <int MODE, typename T, int VEC>
@@ -369,24 +1025,81 @@ void dispatch_main(const Params &P, const Shape &s, int dtype, cudaStream_t st) 
 }
 
 template <typename T, int VEC>
-void finish_nv(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s, cudaStream_t st) {
+void fixup_nv(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s, cudaStream_t st) {
     switch (s.nv) {
-        case 1: launch_finish<T, VEC, 1>(D, partial, out, H, s, st); break;
-        case 2: launch_finish<T, VEC, 2>(D, partial, out, H, s, st); break;
-        default: launch_finish<T, VEC, 4>(D, partial, out, H, s, st); break;
+        case 1: launch_fixup<T, VEC, 1>(D, partial, out, H, s, st); break;
+        case 2: launch_fixup<T, VEC, 2>(D, partial, out, H, s, st); break;
+        default: launch_fixup<T, VEC, 4>(D, partial, out, H, s, st); break;
     }
 }
 
-void dispatch_finish(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s,
-                     int dtype, cudaStream_t st) {
+void dispatch_fixup(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s,
+                    int dtype, cudaStream_t st) {
     if (dtype == AG_F32) {
-        if (s.vec == 4) finish_nv<float, 4>(D, partial, out, H, s, st);
-        else finish_nv<float, 1>(D, partial, out, H, s, st);
+        if (s.vec == 4) fixup_nv<float, 4>(D, partial, out, H, s, st);
+        else fixup_nv<float, 1>(D, partial, out, H, s, st);
     } else {
-        if (s.vec == 8) finish_nv<bf16_t, 8>(D, partial, out, H, s, st);
-        else if (s.vec == 2) finish_nv<bf16_t, 2>(D, partial, out, H, s, st);
-        else finish_nv<bf16_t, 1>(D, partial, out, H, s, st);
+        if (s.vec == 8) fixup_nv<bf16_t, 8>(D, partial, out, H, s, st);
+        else if (s.vec == 2) fixup_nv<bf16_t, 2>(D, partial, out, H, s, st);
+        else fixup_nv<bf16_t, 1>(D, partial, out, H, s, st);
     }
+}
+
+template <typename T, int VEC, int NV, int G>
+void launch_dw_coo_g(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, cudaStream_t st) {
+    constexpr int D = kRingDepth < G ? kRingDepth : G;
+    const size_t smem = size_t(kThreads) * 2 * D * NV * 16;
+    static bool configured = false;
+    if (!configured) {
+        cudaFuncSetAttribute(k_dw_coo<T, VEC, NV, G, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        configured = true;
+    }
+    const int64_t per_warp = 32 / G;
+    const int64_t groups = (g->n_tiles + per_warp - 1) / per_warp * per_warp;
+    const unsigned grid = unsigned((groups + kThreads / G - 1) / (kThreads / G));
+    k_dw_coo<T, VEC, NV, G, D><<<grid, kThreads, smem, st>>>(g->coo_src, g->coo_dst, X, dY, dw, int(g->E), int(H),
+                                                            g->tile_edges, g->n_tiles);
+}
+
+template <typename T, int VEC, int NV>
+void launch_dw_coo_nv(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, const Shape &s,
+                      cudaStream_t st) {
+    switch (s.G) {
+        case 4: launch_dw_coo_g<T, VEC, NV, 4>(g, X, dY, dw, H, st); break;
+        case 8: launch_dw_coo_g<T, VEC, NV, 8>(g, X, dY, dw, H, st); break;
+        case 16: launch_dw_coo_g<T, VEC, NV, 16>(g, X, dY, dw, H, st); break;
+        default: launch_dw_coo_g<T, VEC, NV, 32>(g, X, dY, dw, H, st); break;
+    }
+}
+
+void launch_dw_coo(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, int dtype,
+                   const Shape &s, cudaStream_t st) {
+    if (dtype == AG_F32) {
+        if (s.nv == 1) launch_dw_coo_nv<float, 4, 1>(g, X, dY, dw, H, s, st);
+        else launch_dw_coo_nv<float, 4, 2>(g, X, dY, dw, H, s, st);
+    } else {
+        if (s.nv == 1) launch_dw_coo_nv<bf16_t, 8, 1>(g, X, dY, dw, H, s, st);
+        else launch_dw_coo_nv<bf16_t, 8, 2>(g, X, dY, dw, H, s, st);
+    }
+}
+
+Params base_params(const ag_graph *g, const ag::Direction &D, int64_t H, const Shape &s) {
+    Params P{};
+    P.col = D.col;
+    P.order = D.order;
+    P.nz_rows = D.nz_rows;
+    P.nz_rowptr = D.nz_rowptr;
+    P.tile_nz = D.tile_nz;
+    P.zero_rows = D.zero_rows;
+    P.E = g->E;
+    P.H = H;
+    P.n_nz = D.n_nz;
+    P.n_tiles = g->n_tiles;
+    P.T = g->tile_edges;
+    P.G = s.G;
+    P.log2G = s.log2G;
+    P.col_tiles = s.col_tiles;
+    return P;
 }
 
 int check_call(const ag_graph *g, int64_t H, int dtype, const char *fn) {
@@ -398,8 +1111,8 @@ int check_call(const ag_graph *g, int64_t H, int dtype, const char *fn) {
 }
 
 size_t scratch_needed(const ag_graph *g, int64_t H) {
-    int64_t c = g->dir[0].n_chunks > g->dir[1].n_chunks ? g->dir[0].n_chunks : g->dir[1].n_chunks;
-    return size_t(c) * size_t(H) * 4;
+    if (g->dir[0].n_span == 0 && g->dir[1].n_span == 0) return 0;
+    return size_t(2) * size_t(g->n_tiles) * size_t(H) * 4;
 }
 
 // SpMM over direction d: out = A_w X (d = 0) or A_w^T dY (d = 1).
@@ -409,7 +1122,7 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     if (rc != AG_OK) return rc;
     if (!F || !out || (g->E > 0 && !w)) return fail(AG_ERR_INVALID_ARG, "%s: null w, input or output", fn);
     const ag::Direction &D = g->dir[d];
-    const size_t need = size_t(D.n_chunks) * size_t(H) * 4;
+    const size_t need = D.n_span > 0 ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0;
     if (need > 0 && (!scratch || scratch_bytes < need))
         return fail(AG_ERR_WORKSPACE, "%s: scratch of %zu bytes, need %zu", fn, scratch_bytes, need);
     if (!aligned(scratch, 16)) return fail(AG_ERR_WORKSPACE, "%s: scratch must be 16-byte aligned", fn);
@@ -421,24 +1134,14 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape s = pick_shape(H, dtype, F, out, nullptr);
-    Params P{};
-    P.rows = D.rows;
-    P.chunks = D.chunks;
-    P.col = D.col;
-    P.order = D.order;
+    Params P = base_params(g, D, H, s);
     P.w = w;
     P.F = F;
     P.out = out;
     P.partial = static_cast<float *>(scratch);
-    P.H = H;
-    P.n_chunks = D.n_chunks;
-    P.row_first = D.n_heavy;
-    P.n_items = D.n_chunks + (g->N - D.n_heavy);
-    P.G = s.G;
-    P.log2G = s.log2G;
-    P.col_tiles = s.col_tiles;
-    if (P.n_items > 0) dispatch_main<kSpmm>(P, s, dtype, st);
-    if (D.n_heavy > 0) dispatch_finish(D, P.partial, out, H, s, dtype, st);
+    P.n_zero = g->N - D.n_nz;
+    if (P.n_tiles + P.n_zero > 0) dispatch_main<kSpmm>(P, s, dtype, st);
+    if (D.n_span > 0) dispatch_fixup(D, P.partial, out, H, s, dtype, st);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
@@ -459,22 +1162,67 @@ int sddmm(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H
     const ag::Direction &D = g->dir[1];
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape s = pick_shape(H, dtype, X, dY, nullptr);
-    Params P{};
-    P.rows = D.rows;
-    P.chunks = D.chunks;
-    P.col = D.col;
-    P.order = D.order;
+#if AG_DW_COO
+    if (s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8)) {
+        launch_dw_coo(g, X, dY, dw, H, dtype, s, st);
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return cuda_fail(err, fn);
+        return AG_OK;
+    }
+#endif
+    Params P = base_params(g, D, H, s);
     P.F = dY;
     P.R = X;
     P.dw = dw;
-    P.H = H;
-    P.n_chunks = D.n_chunks;
-    P.row_first = D.n_heavy;
-    P.n_items = D.n_chunks + (D.n_nonempty - D.n_heavy);
-    P.G = s.G;
-    P.log2G = s.log2G;
-    P.col_tiles = s.col_tiles;
-    if (P.n_items > 0) dispatch_main<kSddmm>(P, s, dtype, st);
+    P.n_zero = 0;
+    dispatch_main<kSddmm>(P, s, dtype, st);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    return AG_OK;
+}
+
+// Feature gradient and weight gradient in one walk of the transpose CSR.
+int backward(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw, int64_t H,
+             int dtype, void *scratch, size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs) {
+    int rc = check_call(g, H, dtype, fn);
+    if (rc != AG_OK) return rc;
+    if (!X || !dY || !dX || (g->E > 0 && (!w || !dw)))
+        return fail(AG_ERR_INVALID_ARG, "%s: null w, X, dY, dX or dw", fn);
+    const ag::Direction &D = g->dir[1];
+    const size_t need = D.n_span > 0 ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0;
+    if (need > 0 && (!scratch || scratch_bytes < need))
+        return fail(AG_ERR_WORKSPACE, "%s: scratch of %zu bytes, need %zu", fn, scratch_bytes, need);
+    if (!aligned(scratch, 16)) return fail(AG_ERR_WORKSPACE, "%s: scratch must be 16-byte aligned", fn);
+    if (check_ptrs) {
+        if ((rc = check_device_ptr(X, g->device, "X")) != AG_OK) return rc;
+        if ((rc = check_device_ptr(dY, g->device, "dY")) != AG_OK) return rc;
+        if ((rc = check_device_ptr(dX, g->device, "dX")) != AG_OK) return rc;
+        if (g->E > 0 && (rc = check_device_ptr(w, g->device, "w")) != AG_OK) return rc;
+        if (g->E > 0 && (rc = check_device_ptr(dw, g->device, "dw")) != AG_OK) return rc;
+        if (need > 0 && (rc = check_device_ptr(scratch, g->device, "scratch")) != AG_OK) return rc;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Shape s = pick_shape(H, dtype, X, dY, dX);
+    const bool ring = s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8);
+    // The single walk scatters dw through transpose_order; that only pays when
+    // consecutive positions mostly share dw sectors (a source-sorted COO list).
+    // Otherwise the transpose-CSR SpMM and the COO-order SDDMM (coalesced dw)
+    // are faster.  Both choices give bitwise identical results.
+    const bool single_walk = ring && g->dw_locality >= kSingleWalkLocality;
+    if (!single_walk || g->E == 0) {
+        if ((rc = spmm(g, 1, w, dY, dX, H, dtype, scratch, scratch_bytes, stream, fn, false)) != AG_OK) return rc;
+        return sddmm(g, X, dY, dw, H, dtype, stream, fn, false);
+    }
+    Params P = base_params(g, D, H, s);
+    P.w = w;
+    P.F = dY;
+    P.R = X;
+    P.out = dX;
+    P.dw = dw;
+    P.partial = static_cast<float *>(scratch);
+    P.n_zero = g->N - D.n_nz;
+    dispatch_main<kBoth>(P, s, dtype, st);
+    if (D.n_span > 0) dispatch_fixup(D, P.partial, dX, H, s, dtype, st);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
@@ -508,6 +1256,12 @@ int ag_sddmm_dw(const ag_graph *g, const void *X, const void *dY, float *dw, int
                 void *stream) {
     clear_error();
     return sddmm(g, X, dY, dw, H, dtype, stream, "ag_sddmm_dw", true);
+}
+
+int ag_backward(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw, int64_t H,
+                int dtype, void *scratch, size_t scratch_bytes, void *stream) {
+    clear_error();
+    return backward(g, w, X, dY, dX, dw, H, dtype, scratch, scratch_bytes, stream, "ag_backward", true);
 }
 
 // Staging layout: w | X | dY | Y | dX | dw | scratch, each 256-byte aligned.
@@ -565,9 +1319,9 @@ int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, con
     copy(Y_host, Y, feat, cudaMemcpyDeviceToHost);
     copy(dY, dY_host, feat, cudaMemcpyHostToDevice);
     if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy");
-    if ((rc = spmm(g, 1, w, dY, dX, H, dtype, scratch, scr, stream, "ag_step_host", false)) != AG_OK) return rc;
+    if ((rc = backward(g, w, X, dY, dX, dw, H, dtype, scratch, scr, stream, "ag_step_host", false)) != AG_OK)
+        return rc;
     copy(dX_host, dX, feat, cudaMemcpyDeviceToHost);
-    if ((rc = sddmm(g, X, dY, dw, H, dtype, stream, "ag_step_host", false)) != AG_OK) return rc;
     copy(dw_host, dw, wb, cudaMemcpyDeviceToHost);
     if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy out");
     return AG_OK;

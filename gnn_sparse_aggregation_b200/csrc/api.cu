@@ -41,10 +41,10 @@ int check_device_ptr(const void *p, int device, const char *name) {
     return AG_OK;
 }
 
-int64_t max_chunks(int64_t E) {
-    // sum over split rows of ceil(deg / C) <= E / C + (number of split rows),
-    // and a split row has more than kHeavyThreshold edges
-    return E / kChunkEdges + E / (kHeavyThreshold + 1) + 1;
+int pick_tile_edges(int64_t E) {
+    int T = kMaxTileEdges;
+    while (T > kMinTileEdges && n_tiles_for(E, T) < kFillGroups) T >>= 1;
+    return T;
 }
 
 static size_t scan_tmp_elems(size_t n) {
@@ -69,18 +69,24 @@ bool make_layout(int64_t N, int64_t E, Layout *L) {
         off += align_up(bytes ? bytes : 1);
         return at;
     };
+    const size_t tiles = size_t(n_tiles_for(E, pick_tile_edges(E)));
     for (int d = 0; d < 2; ++d) {
         L->rowptr[d] = take((n + 1) * 4);
         L->col[d] = take(e * 4);
         L->order[d] = take(e * 4);
-        L->rows[d] = take(n * 16);
-        L->chunks[d] = take(size_t(max_chunks(E)) * 16);
+        L->nz_rows[d] = take(n * 4);
+        L->nz_rowptr[d] = take((n + 1) * 4);
+        L->zero_rows[d] = take(n * 4);
+        L->tile_nz[d] = take(tiles * 4);
+        L->spans[d] = take((tiles < n ? tiles : n) * 16);  // a tile boundary cuts at most one row
     }
-    // lowering temporaries (unused after ag_graph_lower returns)
-    L->keys_a = take(m * 4);
-    L->vals_a = take(m * 4);
-    L->keys_b = take(m * 4);
-    L->vals_b = take(m * 4);
+    L->coo_src = take(e * 4);
+    L->coo_dst = take(e * 4);
+    // lowering temporaries (unused after ag_graph_lower returns); +1 for scan totals
+    L->keys_a = take((m + 1) * 4);
+    L->vals_a = take((m + 1) * 4);
+    L->keys_b = take((m + 1) * 4);
+    L->vals_b = take((m + 1) * 4);
     L->hist = take((256 * nblk + 1) * 4);  // +1: the in-place scan writes its total at [n]
     size_t scan_n = 256 * nblk + 1 > n + 1 ? 256 * nblk + 1 : n + 1;
     L->scan_tmp = take(scan_tmp_elems(scan_n) * 4);
@@ -121,17 +127,18 @@ int ag_graph_get_stats(const ag_graph *g, ag_graph_stats *out) {
     out->N = g->N;
     out->E = g->E;
     out->device = g->device;
-    out->chunk_edges = kChunkEdges;
-    out->heavy_threshold = kHeavyThreshold;
+    out->tile_edges = g->tile_edges;
+    out->tiles = g->n_tiles;
     out->max_degree_f = g->dir[0].max_degree;
     out->max_degree_t = g->dir[1].max_degree;
-    out->heavy_rows_f = g->dir[0].n_heavy;
-    out->chunks_f = g->dir[0].n_chunks;
-    out->nonempty_rows_f = g->dir[0].n_nonempty;
-    out->heavy_rows_t = g->dir[1].n_heavy;
-    out->chunks_t = g->dir[1].n_chunks;
-    out->nonempty_rows_t = g->dir[1].n_nonempty;
+    out->nonempty_rows_f = g->dir[0].n_nz;
+    out->spanning_rows_f = g->dir[0].n_span;
+    out->long_spanning_rows_f = g->dir[0].n_span_long;
+    out->nonempty_rows_t = g->dir[1].n_nz;
+    out->spanning_rows_t = g->dir[1].n_span;
+    out->long_spanning_rows_t = g->dir[1].n_span_long;
     out->workspace_bytes_used = g->ws_used;
+    out->dw_locality = g->dw_locality;
     return AG_OK;
 }
 

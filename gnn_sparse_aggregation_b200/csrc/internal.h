@@ -9,27 +9,32 @@
 
 namespace ag {
 
-// Rows with more than kHeavyThreshold edges are split into chunks of
-// kChunkEdges edges; each chunk writes an fp32 partial row to scratch, and a
-// second kernel adds a heavy row's partials in chunk order.
-constexpr int kChunkEdges = 256;
-constexpr int64_t kHeavyThreshold = 256;
+// Per-call kernels walk the CSR in tiles of `tile_edges` consecutive
+// positions (a power of two between kMinTileEdges and kMaxTileEdges, chosen
+// at lowering so that there are enough tiles to fill the GPU).  A row cut by
+// a tile boundary leaves one fp32 partial row per tile, and a second kernel
+// adds a row's partials in tile order.  Rows cut into more than
+// kLongSpanTiles + 1 tiles are added up by a whole CTA.
+constexpr int kMaxTileEdges = 512;
+constexpr int kMinTileEdges = 32;
+constexpr int kFillGroups = 148 * 64;  // tiles wanted: SMs x resident lane groups
+constexpr int kLongSpanTiles = 8;
 
 constexpr size_t kAlign = 256;
 
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 
-// Row schedule of one CSR direction.  `rows` lists every row as
-// {row, csr_begin, csr_end, first_chunk} in order of decreasing degree (ties
-// by ascending row id): the first n_heavy entries are the split rows, then
-// the other non-empty rows, then the empty rows.
+// Schedule of one CSR direction.
 struct Direction {
-    int32_t *rowptr = nullptr;  // [N+1]
-    int32_t *col = nullptr;     // [E] the other endpoint of each CSR position
-    int32_t *order = nullptr;   // [E] CSR position -> COO ordinal
-    int4 *rows = nullptr;       // [N]
-    int4 *chunks = nullptr;     // [n_chunks] {csr_begin, csr_end, row, split-row index}
-    int64_t n_heavy = 0, n_chunks = 0, n_nonempty = 0, max_degree = 0;
+    int32_t *rowptr = nullptr;     // [N+1]
+    int32_t *col = nullptr;        // [E] the other endpoint of each CSR position
+    int32_t *order = nullptr;      // [E] CSR position -> COO ordinal
+    int32_t *nz_rows = nullptr;    // [n_nz] rows with at least one edge, ascending
+    int32_t *nz_rowptr = nullptr;  // [n_nz + 1] first CSR position of each, then E
+    int32_t *zero_rows = nullptr;  // [N - n_nz] rows without edges, ascending
+    int32_t *tile_nz = nullptr;    // [n_tiles] index into nz_rows of the row holding the tile's first position
+    int4 *spans = nullptr;         // [n_span] {row, first tile, last tile, 0}: long spans first
+    int64_t n_nz = 0, n_span = 0, n_span_long = 0, max_degree = 0;
 };
 
 }  // namespace ag
@@ -37,7 +42,15 @@ struct Direction {
 struct ag_graph {
     int device = 0;
     int64_t N = 0, E = 0;
+    int tile_edges = ag::kMaxTileEdges;
+    int64_t n_tiles = 0;
     size_t ws_used = 0;
+    int32_t *coo_src = nullptr;  // [E] copies of the COO endpoints (edge identity)
+    int32_t *coo_dst = nullptr;
+    // fraction of transpose-CSR positions whose COO ordinal shares a 32-byte
+    // dw sector with the previous position's: high when the COO list is
+    // (nearly) sorted by source, ~0 for an arbitrary edge order
+    double dw_locality = 0.0;
     ag::Direction dir[2];  // 0: forward CSR (owned by destination), 1: transpose CSR (by source)
 };
 
@@ -53,11 +66,13 @@ int check_device_ptr(const void *p, int device, const char *name);
 
 // Lowering-time workspace layout (shared by the size query and the lowering).
 struct Layout {
-    size_t rowptr[2], col[2], order[2], rows[2], chunks[2];
+    size_t rowptr[2], col[2], order[2], nz_rows[2], nz_rowptr[2], zero_rows[2], tile_nz[2], spans[2];
+    size_t coo_src, coo_dst;
     size_t keys_a, vals_a, keys_b, vals_b, hist, scan_tmp, aux, counters;
     size_t total;
 };
 bool make_layout(int64_t N, int64_t E, Layout *L);
-int64_t max_chunks(int64_t E);
+int pick_tile_edges(int64_t E);
+inline int64_t n_tiles_for(int64_t E, int T) { return (E + T - 1) / T; }
 
 }  // namespace ag

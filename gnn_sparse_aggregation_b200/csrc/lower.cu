@@ -15,9 +15,10 @@
 //      the scatter ranks equal digits with __match_any_sync inside a warp
 //      and in warp order across the tile, so equal keys keep COO order;
 //   3. rowptr[r] = lower_bound(sorted keys, r), col = other[order];
-//   4. the row schedule: rows sorted by decreasing degree (the same stable
-//      radix sort on maxdeg - deg), rows longer than kHeavyThreshold split
-//      into kChunkEdges-edge chunks.
+//   4. the tile schedule of the per-call kernels: the non-empty rows
+//      compacted (ids and first positions), the empty rows listed, the row
+//      holding the first position of every tile, and the rows cut by a tile
+//      boundary (long ones first).
 #include <cstdio>
 
 #include "internal.h"
@@ -234,53 +235,76 @@ __global__ void k_max_degree(const int32_t *__restrict__ rowptr, int64_t N, int 
     if ((threadIdx.x & 31) == 0 && m > 0) atomicMax(maxdeg, m);
 }
 
-__global__ void k_degree_keys(const int32_t *__restrict__ rowptr, int64_t N, int maxdeg,
-                              int32_t *__restrict__ keys) {
+// flags[r] = 1 if row r has at least one edge
+__global__ void k_nz_flags(const int32_t *__restrict__ rowptr, int64_t N, int32_t *__restrict__ flags) {
     for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < N;
          r += int64_t(gridDim.x) * blockDim.x)
-        keys[r] = maxdeg - (rowptr[r + 1] - rowptr[r]);
+        flags[r] = rowptr[r + 1] > rowptr[r] ? 1 : 0;
 }
 
-// sched is sorted by decreasing degree; count the split rows and non-empty
-// rows (both are prefixes) and the chunks of every split row.
-__global__ void k_sched_counts(const int32_t *__restrict__ sched, const int32_t *__restrict__ rowptr,
-                               int64_t N, int32_t *__restrict__ nch, int *n_heavy, int *n_nonempty) {
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < N;
-         i += int64_t(gridDim.x) * blockDim.x) {
-        const int r = sched[i];
-        const int deg = rowptr[r + 1] - rowptr[r];
-        int next = -1;
-        if (i + 1 < N) {
-            const int r2 = sched[i + 1];
-            next = rowptr[r2 + 1] - rowptr[r2];
+// pos = exclusive scan of the flags (pos[N] = number of non-empty rows).
+__global__ void k_nz_scatter(const int32_t *__restrict__ rowptr, const int32_t *__restrict__ pos, int64_t N,
+                             int64_t E, int32_t *__restrict__ nz_rows, int32_t *__restrict__ nz_rowptr,
+                             int32_t *__restrict__ zero_rows) {
+    for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < N;
+         r += int64_t(gridDim.x) * blockDim.x) {
+        const int i = pos[r];
+        if (rowptr[r + 1] > rowptr[r]) {
+            nz_rows[i] = int32_t(r);
+            nz_rowptr[i] = rowptr[r];
+        } else {
+            zero_rows[r - i] = int32_t(r);
         }
-        nch[i] = deg > kHeavyThreshold ? (deg + kChunkEdges - 1) / kChunkEdges : 0;
-        if (deg > kHeavyThreshold && next <= kHeavyThreshold) *n_heavy = int(i + 1);
-        if (deg > 0 && next <= 0) *n_nonempty = int(i + 1);
+        if (r == N - 1) nz_rowptr[pos[N]] = int32_t(E);
     }
 }
 
-__global__ void k_rows_fill(const int32_t *__restrict__ sched, const int32_t *__restrict__ rowptr,
-                            const int32_t *__restrict__ chunk_off, int64_t N, int64_t n_heavy,
-                            int4 *__restrict__ rows) {
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < N;
+// tile_nz[t] = the non-empty row i with nz_rowptr[i] <= t*T < nz_rowptr[i+1].
+__global__ void k_tile_nz(const int32_t *__restrict__ nz_rowptr, int64_t n_nz, int T,
+                          int32_t *__restrict__ tile_nz) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_nz;
          i += int64_t(gridDim.x) * blockDim.x) {
-        const int r = sched[i];
-        rows[i] = make_int4(r, rowptr[r], rowptr[r + 1], i < n_heavy ? chunk_off[i] : 0);
+        const int64_t b = nz_rowptr[i], e = nz_rowptr[i + 1];
+        for (int64_t t = (b + T - 1) / T; t <= (e - 1) / T; ++t) tile_nz[t] = int32_t(i);
     }
 }
 
-// One warp per split row writes its chunk table entries.
-__global__ void k_chunks_fill(const int4 *__restrict__ rows, int64_t n_heavy, int4 *__restrict__ chunks) {
-    const int64_t h = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (h >= n_heavy) return;
-    const int4 r = rows[h];
-    const int nch = (r.z - r.y + kChunkEdges - 1) / kChunkEdges;
-    for (int j = lane; j < nch; j += 32) {
-        const int b = r.y + j * kChunkEdges;
-        chunks[int64_t(r.w) + j] = make_int4(b, min(b + kChunkEdges, r.z), r.x, int(h));
+// Rows whose first and last edge fall in different tiles; `lng` marks those
+// that cross more than kLongSpanTiles tile boundaries.
+__global__ void k_span_flags(const int32_t *__restrict__ nz_rowptr, int64_t n_nz, int T,
+                             int32_t *__restrict__ lng, int32_t *__restrict__ shrt) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_nz;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t ta = nz_rowptr[i] / T, tb = (int64_t(nz_rowptr[i + 1]) - 1) / T;
+        const bool span = ta != tb;
+        const bool is_long = span && tb - ta > kLongSpanTiles;
+        lng[i] = is_long ? 1 : 0;
+        shrt[i] = (span && !is_long) ? 1 : 0;
     }
+}
+
+__global__ void k_span_scatter(const int32_t *__restrict__ nz_rows, const int32_t *__restrict__ nz_rowptr,
+                               int64_t n_nz, int T, const int32_t *__restrict__ lpos,
+                               const int32_t *__restrict__ spos, int64_t n_long, int4 *__restrict__ spans) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_nz;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t ta = nz_rowptr[i] / T, tb = (int64_t(nz_rowptr[i + 1]) - 1) / T;
+        if (ta == tb) continue;
+        const int4 v = make_int4(nz_rows[i], int(ta), int(tb), 0);
+        if (tb - ta > kLongSpanTiles) spans[lpos[i]] = v;
+        else spans[n_long + spos[i]] = v;
+    }
+}
+
+// Number of positions p > 0 whose ordinal lies in the same 8-ordinal
+// (32-byte) sector as the ordinal at p - 1.
+__global__ void k_sector_runs(const int32_t *__restrict__ order, int64_t n, unsigned long long *count) {
+    unsigned c = 0;
+    for (int64_t p = 1 + blockIdx.x * int64_t(blockDim.x) + threadIdx.x; p < n;
+         p += int64_t(gridDim.x) * blockDim.x)
+        c += (order[p] >> 3) == (order[p - 1] >> 3) ? 1u : 0u;
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if ((threadIdx.x & 31) == 0 && c) atomicAdd(count, (unsigned long long)c);
 }
 
 inline unsigned grid_for(int64_t n, int threads, int64_t cap = 148 * 64) {
@@ -407,14 +431,26 @@ extern "C" int ag_graph_lower(const int32_t *src, const int32_t *dst, int64_t N,
     g.N = N;
     g.E = E;
     g.ws_used = L.total;
+    g.tile_edges = pick_tile_edges(E);
+    g.n_tiles = n_tiles_for(E, g.tile_edges);
+    g.coo_src = I(L.coo_src);
+    g.coo_dst = I(L.coo_dst);
+    if (E > 0) {
+        err = cudaMemcpyAsync(g.coo_src, src, size_t(E) * 4, cudaMemcpyDeviceToDevice, s);
+        if (err == cudaSuccess) err = cudaMemcpyAsync(g.coo_dst, dst, size_t(E) * 4, cudaMemcpyDeviceToDevice, s);
+        if (err != cudaSuccess) return cuda_fail(err, "ag_graph_lower: edge copies");
+    }
     const int key_bits = bit_length(N - 1);
     for (int d = 0; d < 2; ++d) {
         Direction &D = g.dir[d];
         D.rowptr = I(L.rowptr[d]);
         D.col = I(L.col[d]);
         D.order = I(L.order[d]);
-        D.rows = reinterpret_cast<int4 *>(ws + L.rows[d]);
-        D.chunks = reinterpret_cast<int4 *>(ws + L.chunks[d]);
+        D.nz_rows = I(L.nz_rows[d]);
+        D.nz_rowptr = I(L.nz_rowptr[d]);
+        D.zero_rows = I(L.zero_rows[d]);
+        D.tile_nz = I(L.tile_nz[d]);
+        D.spans = reinterpret_cast<int4 *>(ws + L.spans[d]);
         const int32_t *key = d == 0 ? dst : src;
         const int32_t *other = d == 0 ? src : dst;
 
@@ -423,32 +459,45 @@ extern "C" int ag_graph_lower(const int32_t *src, const int32_t *dst, int64_t N,
         k_rowptr_search<<<grid_for(N + 1, 256), 256, 0, s>>>(sorted, E, N, D.rowptr);
         if (E > 0) k_gather<<<grid_for(E, 256), 256, 0, s>>>(D.order, other, E, D.col);
 
-        // 4. schedule: rows by decreasing degree
-        cudaMemsetAsync(counters, 0, 8 * sizeof(int), s);
+        // 4. tile schedule
+        err = cudaMemsetAsync(counters, 0, 8 * sizeof(int), s);
+        if (err != cudaSuccess) return cuda_fail(err, "cudaMemsetAsync");
         k_max_degree<<<grid_for(N, 256), 256, 0, s>>>(D.rowptr, N, counters + 1);
-        if ((rc = sync_read("ag_graph_lower: degrees")) != AG_OK) return rc;
-        const int maxdeg = host_counters[1];
-        D.max_degree = maxdeg;
-        k_degree_keys<<<grid_for(N, 256), 256, 0, s>>>(D.rowptr, N, maxdeg, t.aux);
-        // The radix passes ping-pong through keys_a/b and vals_a/b and read
-        // their keys from aux, so the sorted row ids go to rows[] (16 bytes
-        // per row, not yet written) and are then copied to keys_b, because
-        // rows[] is filled from them below.
-        int32_t *sched_out = reinterpret_cast<int32_t *>(D.rows);
-        radix_sort(t.aux, nullptr, N, bit_length(maxdeg), sched_out, t, s);
-        int32_t *sched = t.keys_b;
-        cudaMemcpyAsync(sched, sched_out, size_t(N) * 4, cudaMemcpyDeviceToDevice, s);
-        k_sched_counts<<<grid_for(N, 256), 256, 0, s>>>(sched, D.rowptr, N, t.vals_a,
-                                                        counters + 2, counters + 3);
-        exclusive_scan(t.vals_a, t.aux, N, t.scan, s);  // chunk offsets; aux[N] = total
-        cudaMemcpyAsync(counters + 4, t.aux + N, sizeof(int), cudaMemcpyDeviceToDevice, s);
-        if ((rc = sync_read("ag_graph_lower: schedule")) != AG_OK) return rc;
-        D.n_heavy = host_counters[2];
-        D.n_nonempty = host_counters[3];
-        D.n_chunks = host_counters[4];
-        k_rows_fill<<<grid_for(N, 256), 256, 0, s>>>(sched, D.rowptr, t.aux, N, D.n_heavy, D.rows);
-        if (D.n_heavy > 0)
-            k_chunks_fill<<<unsigned((D.n_heavy * 32 + 255) / 256), 256, 0, s>>>(D.rows, D.n_heavy, D.chunks);
+        k_nz_flags<<<grid_for(N, 256), 256, 0, s>>>(D.rowptr, N, t.vals_a);
+        exclusive_scan(t.vals_a, t.aux, N, t.scan, s);  // aux[N] = non-empty rows
+        k_nz_scatter<<<grid_for(N, 256), 256, 0, s>>>(D.rowptr, t.aux, N, E, D.nz_rows, D.nz_rowptr,
+                                                      D.zero_rows);
+        cudaMemcpyAsync(counters + 2, t.aux + N, sizeof(int), cudaMemcpyDeviceToDevice, s);
+        if ((rc = sync_read("ag_graph_lower: rows")) != AG_OK) return rc;
+        D.max_degree = host_counters[1];
+        D.n_nz = host_counters[2];
+        if (D.n_nz > 0) {
+            k_tile_nz<<<grid_for(D.n_nz, 256), 256, 0, s>>>(D.nz_rowptr, D.n_nz, g.tile_edges, D.tile_nz);
+            k_span_flags<<<grid_for(D.n_nz, 256), 256, 0, s>>>(D.nz_rowptr, D.n_nz, g.tile_edges,
+                                                              t.keys_a, t.keys_b);
+            exclusive_scan(t.keys_a, t.vals_a, D.n_nz, t.scan, s);  // long spans
+            exclusive_scan(t.keys_b, t.vals_b, D.n_nz, t.scan, s);  // other spans
+            cudaMemcpyAsync(counters + 3, t.vals_a + D.n_nz, sizeof(int), cudaMemcpyDeviceToDevice, s);
+            cudaMemcpyAsync(counters + 4, t.vals_b + D.n_nz, sizeof(int), cudaMemcpyDeviceToDevice, s);
+            if ((rc = sync_read("ag_graph_lower: spans")) != AG_OK) return rc;
+            D.n_span_long = host_counters[3];
+            D.n_span = host_counters[3] + host_counters[4];
+            if (D.n_span > 0)
+                k_span_scatter<<<grid_for(D.n_nz, 256), 256, 0, s>>>(D.nz_rows, D.nz_rowptr, D.n_nz,
+                                                                    g.tile_edges, t.vals_a, t.vals_b,
+                                                                    D.n_span_long, D.spans);
+        }
+    }
+    // locality of the transpose order, for ag_backward's choice of walk
+    if (E > 1) {
+        unsigned long long *cnt = reinterpret_cast<unsigned long long *>(counters + 8);
+        cudaMemsetAsync(cnt, 0, sizeof *cnt, s);
+        k_sector_runs<<<grid_for(E, 256), 256, 0, s>>>(g.dir[1].order, E, cnt);
+        unsigned long long host_cnt = 0;
+        err = cudaMemcpyAsync(&host_cnt, cnt, sizeof host_cnt, cudaMemcpyDeviceToHost, s);
+        if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+        if (err != cudaSuccess) return cuda_fail(err, "ag_graph_lower: locality");
+        g.dw_locality = double(host_cnt) / double(E - 1);
     }
     err = cudaGetLastError();
     if (err == cudaSuccess) err = cudaStreamSynchronize(s);

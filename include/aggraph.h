@@ -73,14 +73,17 @@ typedef enum ag_status {
 /* Schedule facts of a lowered graph, for inspection and tests. */
 typedef struct ag_graph_stats {
     int64_t N, E;
-    int32_t device;           /* CUDA ordinal the graph was lowered on */
-    int32_t chunk_edges;      /* heavy rows are split into chunks of this many edges */
-    int64_t heavy_threshold;  /* rows with more in-edges than this are split */
-    int64_t max_degree_f;     /* largest in-degree (forward CSR row length) */
-    int64_t max_degree_t;     /* largest out-degree (transpose CSR row length) */
-    int64_t heavy_rows_f, chunks_f, nonempty_rows_f;
-    int64_t heavy_rows_t, chunks_t, nonempty_rows_t;
+    int32_t device;             /* CUDA ordinal the graph was lowered on */
+    int32_t tile_edges;         /* per-call kernels walk the CSR in tiles of this many positions */
+    int64_t tiles;              /* ceil(E / tile_edges) */
+    int64_t max_degree_f;       /* largest in-degree (forward CSR row length) */
+    int64_t max_degree_t;       /* largest out-degree (transpose CSR row length) */
+    int64_t nonempty_rows_f;    /* rows with at least one in-edge */
+    int64_t spanning_rows_f;    /* rows cut by a tile boundary (summed from per-tile partials) */
+    int64_t long_spanning_rows_f; /* of those, rows cut into more than 9 tiles */
+    int64_t nonempty_rows_t, spanning_rows_t, long_spanning_rows_t; /* same, transpose CSR */
     size_t workspace_bytes_used;
+    double dw_locality;         /* share of transpose-CSR neighbours whose COO ordinals share a dw sector */
 } ag_graph_stats;
 
 /*
@@ -133,9 +136,9 @@ AG_API int ag_graph_get_stats(const ag_graph *g, ag_graph_stats *out);
 
 /*
  * Device scratch, in bytes, that ag_spmm_fwd / ag_spmm_dx / ag_step_host need
- * for feature width H: fp32 partial rows for the chunks of heavy rows
- * (chunks x H x 4 bytes, the larger of the two directions).  0 when the graph
- * has no heavy row.  This is O(E / chunk_edges * H), never E x H.
+ * for feature width H: two fp32 partial rows per tile for the rows that a
+ * tile boundary cuts (2 x tiles x H x 4 bytes), 0 when no row is cut.  This
+ * is O(E / tile_edges * H), never E x H.
  */
 AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
 
@@ -151,8 +154,8 @@ AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
  *   Y        device [N, H] of dtype, fully written; rows without in-edges are 0
  *   scratch  device buffer of ag_spmm_scratch_bytes(g, H) bytes (NULL if 0),
  *            16-byte aligned; its contents are scratch only
- * Heavy rows are summed in fixed chunk order, so results are bitwise
- * reproducible.  Errors: AG_ERR_INVALID_ARG, AG_ERR_SHAPE (H < 1 or N*H too
+ * Rows cut by tile boundaries are summed in fixed tile order, so results are
+ * bitwise reproducible.  Errors: AG_ERR_INVALID_ARG, AG_ERR_SHAPE (H < 1 or N*H too
  * large), AG_ERR_DTYPE, AG_ERR_DEVICE, AG_ERR_WORKSPACE, AG_ERR_CUDA.
  */
 AG_API int ag_spmm_fwd(const ag_graph *g, const float *w, const void *X, void *Y, int64_t H,
@@ -182,9 +185,32 @@ AG_API int ag_sddmm_dw(const ag_graph *g, const void *X, const void *dY, float *
                 int dtype, void *stream);
 
 /*
+ * Feature gradient and weight gradient in one pass over the transpose CSR:
+ * dX = A_w^T dY and dw_e = dot(X[src_e], dY[dst_e]).  Both follow the
+ * definitions of "Edge order is explicit" (tinymesh "Weighted aggregation
+ * experiment"); the fusion is this library's: every dY row gathered for an
+ * edge feeds both the dX row of the edge's source and the edge's dot
+ * product, so dY is gathered once for both gradients instead of twice.
+ * Results are bitwise identical to ag_spmm_dx followed by ag_sddmm_dw.  The
+ * single walk writes dw through transpose_order, which costs a 32-byte
+ * sector per edge when the COO order is unrelated to the source order; so it
+ * is used only when ag_graph_stats.dw_locality >= 0.5 (a source-sorted COO
+ * list), and otherwise this call runs the two separate passes.
+ *
+ *   w        device float [E], COO order
+ *   X, dY    device [N, H] of dtype
+ *   dX       device [N, H] of dtype, fully written
+ *   dw       device float [E], COO order
+ *   scratch  as ag_spmm_dx (ag_spmm_scratch_bytes(g, H) bytes)
+ * Errors as ag_spmm_fwd.
+ */
+AG_API int ag_backward(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw,
+                       int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
  * One whole aggregation step from HOST buffers: copies w, X and dY to the
- * device staging area, runs forward, feature gradient and weight gradient,
- * and copies Y, dX and dw back, all enqueued on `stream` in that order.
+ * device staging area, runs the forward pass and the fused backward pass
+ * (ag_backward), and copies Y, dX and dw back, all enqueued on `stream`.
  *
  *   *_host   host buffers (page-locked memory is needed for the copies to be
  *            asynchronous); w_host/dw_host may be NULL when E == 0

@@ -50,6 +50,18 @@ def run_path(g, wl, stream=None):
     return Y, dX, dw
 
 
+def bits(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+
+def check_fused_backward(g, wl, dX, dw):
+    """ag_backward must reproduce ag_spmm_dx and ag_sddmm_dw bit for bit."""
+    fdX, fdw = g.backward(wl.w, wl.X, wl.dY)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(fdX), bits(dX)), "fused dX differs from ag_spmm_dx"
+    assert torch.equal(bits(fdw), bits(dw)), "fused dw differs from ag_sddmm_dw"
+
+
 def oracle_full(wl):
     import oracle
     src, dst = host(wl.src), host(wl.dst)
@@ -68,6 +80,7 @@ def check_full(g, wl, what=""):
     assert_within(Y, rY, bY, tol, f"{what} fwd")
     assert_within(dX, rX, bX, tol, f"{what} dX")
     assert_within(dw, rw, bw, TOL_DW, f"{what} dw")
+    check_fused_backward(g, wl, dX, dw)
     return Y, dX, dw
 
 

@@ -92,18 +92,19 @@ def test_config_no_edge_feature_temporary(config):
     bounded by node state, edge state or row pointers)."""
     wl, g = config
     s = g.stats
-    assert g.scratch_bytes(wl.H) == 4 * wl.H * max(s["chunks_f"], s["chunks_t"])
-    assert g.scratch_bytes(wl.H) < wl.E * wl.H * 4 // 16
+    spans = s["spanning_rows_f"] + s["spanning_rows_t"]
+    assert g.scratch_bytes(wl.H) == (2 * 4 * wl.H * s["tiles"] if spans else 0)
+    assert g.scratch_bytes(wl.H) <= wl.E * wl.H * 4 // 8
     assert g.workspace.numel() < 80 * (wl.N + wl.E) + (1 << 16)
 
 
-def test_rmat16_has_split_rows(config):
+def test_rmat16_has_long_spanning_rows(config):
     wl, g = config
     if wl.name != "rmat16":
-        pytest.skip("split rows are exercised by the R-MAT graph")
+        pytest.skip("rows cut into many tiles are exercised by the R-MAT graph")
     s = g.stats
-    assert s["heavy_rows_f"] > 0 and s["chunks_f"] > s["heavy_rows_f"]
-    assert s["heavy_rows_t"] > 0 and s["max_degree_f"] > 5000
+    assert s["long_spanning_rows_f"] > 0 and s["spanning_rows_f"] > s["long_spanning_rows_f"]
+    assert s["long_spanning_rows_t"] > 0 and s["max_degree_f"] > 5000
 
 
 # ----------------------------------------------------------------------------- edge cases
@@ -115,7 +116,7 @@ def graph(agb, N, src, dst, H, dtype=torch.float32, seed=5, wdist="normal"):
 
 def skewed_edges(N=3000, E=40000, seed=3):
     """Random edges plus a hub with 3,000 in-edges and one with 2,500 out-edges
-    (both split), duplicates, self-loops and many empty rows."""
+    (both cut into many tiles), duplicates, self-loops and many empty rows."""
     rng = np.random.default_rng(seed)
     src = rng.integers(0, N // 3, E)
     dst = rng.integers(0, N // 2, E)
@@ -132,7 +133,7 @@ def skewed_edges(N=3000, E=40000, seed=3):
 def test_widths_and_split_rows(agb, H, dtype):
     N, src, dst = skewed_edges()
     wl, g = graph(agb, N, src, dst, H, dtype)
-    assert g.stats["heavy_rows_f"] >= 1 and g.stats["heavy_rows_t"] >= 1
+    assert g.stats["long_spanning_rows_f"] >= 1 and g.stats["long_spanning_rows_t"] >= 1
     check_full(g, wl, f"H={H} {dtype}")
 
 
@@ -218,6 +219,34 @@ def test_paired_permutation_keeps_outputs(agb):
     assert torch.equal(dw2, dw[perm])       # each edge's dot is computed the same way
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("H", [16, 64, 128, 256])
+def test_single_walk_backward_on_source_sorted_coo(agb, H, dtype):
+    """A COO list sorted by source makes dw writes sector-local, so ag_backward
+    takes the single walk; it must still equal the oracle and the separate
+    passes bit for bit (check_full compares both)."""
+    N, src, dst = skewed_edges()
+    order = np.argsort(src, kind="stable")
+    wl, g = graph(agb, N, src[order], dst[order], H, dtype)
+    assert g.stats["dw_locality"] >= 0.5
+    check_full(g, wl, f"sorted H={H} {dtype}")
+
+
+def test_single_walk_backward_rmat18_sorted(agb):
+    src, dst = workloads.rmat_edges(18, 16, seed=4)
+    order = torch.argsort(src.long() * (1 << 18) + dst.long())
+    wl, g = graph(agb, 1 << 18, src[order].numpy(), dst[order].numpy(), 128, torch.bfloat16)
+    assert g.stats["dw_locality"] >= 0.5
+    check_full(g, wl, "rmat18 sorted")
+
+
+def test_random_order_has_low_locality(config):
+    wl, g = config
+    if wl.name == "twohop":
+        pytest.skip("the sampled block lists edges grouped by sampler")
+    assert g.stats["dw_locality"] < 0.5
+
+
 # ----------------------------------------------------------------------------- API behaviour
 
 def test_non_default_stream(agb):
@@ -264,7 +293,7 @@ def test_errors_are_reported_not_launched(agb):
     # unknown dtype code, bad width
     assert L.ag_spmm_fwd(g.handle, p(wl.w), p(wl.X), p(Y), 8, 7, sp, sn, None) == 3
     assert L.ag_spmm_dx(g.handle, p(wl.w), p(wl.dY), p(Y), 0, 0, sp, sn, None) == 2
-    # scratch too small for the split rows
+    # scratch too small for the rows cut by tile boundaries
     N2, s2, d2 = skewed_edges(N=3000, E=1000)
     wl2, g2 = graph(agb, N2, s2, d2, 8)
     need = g2.scratch_bytes(8)

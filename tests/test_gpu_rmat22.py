@@ -36,7 +36,8 @@ def test_rmat22_shape_and_schedule(big):
     wl, g, _ = big
     assert (wl.N, wl.E, wl.H, wl.feature_dtype) == (1 << 22, 1 << 26, 128, torch.bfloat16)
     s = g.stats
-    assert s["heavy_rows_f"] > 1000 and s["max_degree_f"] > 100_000
+    assert s["tile_edges"] == 512 and s["tiles"] == wl.E // 512
+    assert s["long_spanning_rows_f"] > 100 and s["max_degree_f"] > 100_000
     assert 0 < s["nonempty_rows_f"] < wl.N
 
 
@@ -69,7 +70,7 @@ def test_rmat22_sampled_rows_and_edges(big, host_inputs):
     ref, bound = oracle.spmm_rows(src, dst, wl.N, w, dY, rows_t, by_source=True, with_bound=True)
     assert_within(dX[torch.from_numpy(rows_t).long().cuda()], ref, bound, tol, "rmat22 dX rows")
     edges = np.unique(rng.integers(0, wl.E, 300_000))
-    # and every edge of the heaviest source row (it is split into chunks)
+    # and every edge of the heaviest source row (it is cut into many tiles)
     rp = arr["rowptr_t"].cpu().numpy().astype(np.int64)
     hub = int(np.argmax(np.diff(rp)))
     hub_edges = arr["transpose_order"][rp[hub]:rp[hub + 1]].cpu().numpy()
@@ -89,6 +90,12 @@ def test_rmat22_adjoint_identity(big):
     assert abs(a - c) <= 1e-2 * scale
     assert abs(b - c) <= 1e-2 * scale
     assert np.isfinite([a, b, c]).all()
+
+
+def test_rmat22_fused_backward_matches(big):
+    from tests.gpu_helpers import check_fused_backward
+    wl, g, (Y, dX, dw) = big
+    check_fused_backward(g, wl, dX, dw)
 
 
 def test_rmat22_bitwise_reproducible(big):

@@ -174,8 +174,10 @@ def twohop_edges(n_seeds: int, fanouts, n_global: int, seed: int):
 
 # ----------------------------------------------------------------------------- configs
 
-def make(name: str, seed: int = 1, device="cpu") -> Workload:
-    """One of the five configurations, all tensors on `device`."""
+def make(name: str, seed: int = 1, device="cpu", rmat_scale: int | None = None) -> Workload:
+    """One of the five configurations, all tensors on `device`.  rmat_scale
+    overrides the R-MAT scale of "rmat16"/"rmat22" (same edge factor, width
+    and dtypes) for smaller profiling cases."""
     dev = torch.device(device)
     s = int(seed) * 1000
     if name == "uniform":
@@ -187,6 +189,8 @@ def make(name: str, seed: int = 1, device="cpu") -> Workload:
         N, E = 20000, int(src.shape[0])
     elif name in ("rmat16", "rmat22"):
         scale = 16 if name == "rmat16" else 22
+        if rmat_scale is not None:
+            scale = int(rmat_scale)
         H, wdist = 128, "normal"
         fdt = torch.float32 if name == "rmat16" else torch.bfloat16
         src, dst = rmat_edges(scale, 16, s + 1, dev)
