@@ -78,6 +78,9 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_spmm_dx.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_sddmm_dw.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
     handle.ag_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_spmm_fwd_static_scratch.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
+    handle.ag_spmm_static_scratch_capacity.argtypes = []
+    handle.ag_spmm_static_scratch_capacity.restype = _SZ
     handle.ag_step_staging_bytes.argtypes = [_P, _I64, _I]
     handle.ag_step_staging_bytes.restype = _SZ
     handle.ag_step_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
@@ -87,7 +90,7 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_status_string.argtypes = [_I]
     handle.ag_status_string.restype = ctypes.c_char_p
     for name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
-                 "ag_sddmm_dw", "ag_backward", "ag_step_host", "ag_abi_version"):
+                 "ag_sddmm_dw", "ag_backward", "ag_spmm_fwd_static_scratch", "ag_step_host", "ag_abi_version"):
         getattr(handle, name).restype = _I
     return handle
 
@@ -303,6 +306,23 @@ def ag_backward(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, dX
     _check(lib.ag_backward(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(dX), _ptr(dw), H, code, _ptr(scr),
                            0 if scr is None else scr.numel(), _stream(g.device, stream)))
     return dX, dw
+
+
+def ag_spmm_fwd_static_scratch(g: Graph, w: torch.Tensor, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """Y = A_w X like ag_spmm_fwd, using the library's built-in scratch array
+    instead of a scratch tensor, for callers that cannot allocate device
+    memory at call time (see include/aggraph.h for the limits)."""
+    _check_edge_vec(g, "w", w)
+    code = _check_feat(g, "X", X)
+    if out is None:
+        out = torch.empty_like(X)
+    elif out.shape != X.shape or out.dtype != X.dtype:
+        raise AggraphError(2, "Y must match X in shape and dtype")
+    else:
+        _need_cuda("Y", out)
+    _check(lib.ag_spmm_fwd_static_scratch(g.handle, _ptr(w), _ptr(X), _ptr(out), X.shape[1], code,
+                                          _stream(g.device, stream)))
+    return out
 
 
 def ag_step_staging_bytes(g: Graph, H: int, dtype: torch.dtype) -> int:

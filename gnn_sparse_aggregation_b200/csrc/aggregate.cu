@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 
 #include <climits>
+#include <mutex>
 
 #include "internal.h"
 
@@ -1325,6 +1326,67 @@ int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, con
     copy(dw_host, dw, wb, cudaMemcpyDeviceToHost);
     if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy out");
     return AG_OK;
+}
+
+
+// ---------------------------------------------------------------------------- forward without caller scratch
+
+}  // extern "C"
+
+// Built-in scratch for ag_spmm_fwd_static_scratch: a fixed device array that
+// every GPU loading this library holds until the process exits.  In host code
+// the name g_static_scratch only stands in for the symbol; its device address
+// comes from cudaGetSymbolAddress below.
+static constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up once
+// per device; the host-side name is only a stand-in for the symbol).
+int static_scratch(int device, void **out) {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[device]) {
+        void *p = nullptr;
+        cudaError_t err = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (err != cudaSuccess) return ag::cuda_fail(err, "ag_spmm_fwd_static_scratch: cudaGetSymbolAddress");
+        g_static_ptr[device] = p;
+    }
+    *out = g_static_ptr[device];
+    return AG_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t ag_spmm_static_scratch_capacity(void) { return kStaticScratchBytes; }
+
+int ag_spmm_fwd_static_scratch(const ag_graph *g, const float *w, const void *X, void *Y, int64_t H, int dtype,
+                               void *stream) {
+    clear_error();
+    if (!g) return fail(AG_ERR_INVALID_ARG, "ag_spmm_fwd_static_scratch: null graph");
+    if (H < 1) return fail(AG_ERR_SHAPE, "ag_spmm_fwd_static_scratch: H=%lld", (long long)H);
+    const size_t need = g->dir[0].n_span > 0 ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0;
+    if (need > kStaticScratchBytes)
+        return fail(AG_ERR_WORKSPACE,
+                    "ag_spmm_fwd_static_scratch: this graph needs %zu bytes of scratch at H=%lld, more than the "
+                    "built-in %zu; use ag_spmm_fwd with caller scratch",
+                    need, (long long)H, kStaticScratchBytes);
+    int device = -1;
+    cudaError_t err = cudaGetDevice(&device);
+    if (err != cudaSuccess) return cuda_fail(err, "ag_spmm_fwd_static_scratch: cudaGetDevice");
+    if (device != g->device)
+        return fail(AG_ERR_DEVICE, "ag_spmm_fwd_static_scratch: current device %d, graph is on device %d", device,
+                    g->device);
+    if (device < 0 || device >= kMaxDevices)
+        return fail(AG_ERR_DEVICE, "ag_spmm_fwd_static_scratch: device %d out of range", device);
+    void *scratch = nullptr;
+    int rc = static_scratch(device, &scratch);
+    if (rc != AG_OK) return rc;
+    return spmm(g, 0, w, X, Y, H, dtype, scratch, kStaticScratchBytes, stream, "ag_spmm_fwd_static_scratch", true);
 }
 
 }  // extern "C"

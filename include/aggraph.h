@@ -223,6 +223,38 @@ AG_API int ag_step_host(const ag_graph *g, const float *w_host, const void *X_ho
                  const void *dY_host, void *Y_host, void *dX_host, float *dw_host,
                  int64_t H, int dtype, void *staging, size_t staging_bytes, void *stream);
 
+/*
+ * Forward aggregation without caller scratch (no counterpart on the pages:
+ * an interface addition of this library).
+ *
+ * Same result as ag_spmm_fwd, for callers that cannot allocate device memory
+ * when they call -- for example code that runs while a framework owns the
+ * allocator (allocating behind its back can fail or fragment its pool),
+ * latency-critical paths where cudaMalloc and cudaFree may synchronize the
+ * device, or plug-in hooks that are handed only their input and output
+ * buffers.  The partial rows of rows cut by tile boundaries go to a fixed
+ * device array built into the library instead of caller scratch.
+ *
+ *   - The built-in array holds ag_spmm_static_scratch_capacity() bytes
+ *     (16 MiB) on every GPU that loads the library, until the process exits.
+ *     A graph that needs more (2 x tiles x H x 4 bytes when a row is cut by
+ *     a tile boundary) is rejected with AG_ERR_WORKSPACE; nothing is launched.
+ *   - The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ *     library routine).  Its first call on a device looks up the array's
+ *     device address there (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.  Call it with the graph's device current
+ *     (AG_ERR_DEVICE otherwise).
+ *   - All calls share the one array: calls whose work overlaps on the GPU
+ *     (different streams, different host threads) race and must be ordered
+ *     by the caller.  The array keeps the previous call's contents; no part
+ *     of it has to start at zero, because every partial row a call reads is
+ *     written earlier in the same call.
+ * Arguments and other errors as ag_spmm_fwd.
+ */
+AG_API int ag_spmm_fwd_static_scratch(const ag_graph *g, const float *w, const void *X, void *Y, int64_t H,
+                                      int dtype, void *stream);
+AG_API size_t ag_spmm_static_scratch_capacity(void);
+
 /* Releases the host handle (the caller frees the workspace). NULL is a no-op. */
 AG_API void ag_graph_free(ag_graph *g);
 
