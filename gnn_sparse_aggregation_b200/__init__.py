@@ -76,7 +76,7 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_spmm_scratch_bytes.restype = _SZ
     handle.ag_spmm_fwd.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_spmm_dx.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
-    handle.ag_sddmm_dw.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
+    handle.ag_sddmm_dw.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_spmm_fwd_static_scratch.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
     handle.ag_spmm_static_scratch_capacity.argtypes = []
@@ -177,7 +177,7 @@ class Graph:
         return int(lib.ag_spmm_scratch_bytes(self.handle, H))
 
     def scratch(self, H: int) -> torch.Tensor | None:
-        """Device scratch for the rows cut by tile boundaries at width H (allocated once per H)."""
+        """Device scratch of the per-call functions at width H (allocated once per H)."""
         n = self.scratch_bytes(H)
         if n == 0:
             return None
@@ -279,8 +279,9 @@ def ag_sddmm_dw(g: Graph, X: torch.Tensor, dY: torch.Tensor, out=None, stream=No
         out = torch.empty(g.E, dtype=torch.float32, device=g.device)
     else:
         _check_edge_vec(g, "dw", out)
-    _check(lib.ag_sddmm_dw(g.handle, _ptr(X), _ptr(dY), _ptr(out), X.shape[1], code,
-                           _stream(g.device, stream)))
+    scr = g.scratch(X.shape[1])
+    _check(lib.ag_sddmm_dw(g.handle, _ptr(X), _ptr(dY), _ptr(out), X.shape[1], code, _ptr(scr),
+                           0 if scr is None else scr.numel(), _stream(g.device, stream)))
     return out
 
 

@@ -36,10 +36,20 @@ namespace {
 #define AG_RING_L1 0      // 1: ring copies also allocate in L1 (cp.async.ca), 0: L2 only (.cg)
 #endif
 #ifndef AG_W_STREAM
-#define AG_W_STREAM 1     // 1: weight gathers are loaded evict-first (no reuse to keep in L2)
+#define AG_W_STREAM 0     // 1: weight lookups loaded evict-first; 0: normal caching (the bucketed
+                          // weights of a window are reused from L2 by the window's tiles)
 #endif
 #ifndef AG_DW_COO
-#define AG_DW_COO 1       // 1: weight gradient walks COO order (coalesced dw, two gathers per edge)
+#define AG_DW_COO 0       // 1: standalone weight gradient walks COO order (two gathers per edge)
+#endif
+#ifndef AG_FFMA2
+#define AG_FFMA2 0        // 1: packed fp32x2 FMAs in the ring SpMM (0: scalar fmaf, fewer register moves)
+#endif
+#ifndef AG_RING_STEP
+#define AG_RING_STEP 1    // positions per cp.async wait/commit in the ring SpMM (1 or 2)
+#endif
+#ifndef AG_BUCKET_STAGED
+#define AG_BUCKET_STAGED 1  // 1: weight regrouping passes stage a chunk in shared memory (coalesced)
 #endif
 #ifndef AG_MAX_LANES
 #define AG_MAX_LANES 16   // lanes that share one row (fewer lanes: more 16-byte vectors per lane)
@@ -49,7 +59,6 @@ constexpr int kThreads = 256;
 constexpr int kUnroll = 4;     // gathered rows in flight per lane (register path)
 constexpr int kMinBlocks = 4;  // resident CTAs per SM the register path is compiled for
 constexpr int kRingDepth = AG_RING_DEPTH;
-constexpr double kSingleWalkLocality = 0.5;  // see backward()
 
 enum Mode { kSpmm = 1, kSddmm = 2, kBoth = 3 };  // kBoth: feature and weight gradient in one walk
 
@@ -125,8 +134,9 @@ __device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
     Vec<T, VEC>::unpack(Vec<T, VEC>::load_raw(p), v);
 }
 
-// A weight gathered through edge_order: one 4-byte use per 32-byte sector,
-// with no reuse worth keeping in L2.
+// A weight looked up through the bucketed layout: each 128-byte line of a
+// window is used by about 32 positions of that window's tiles, so it is kept
+// in L2 with the default policy.
 __device__ __forceinline__ float load_w(const float *p) {
 #if AG_W_STREAM
     return __ldcs(p);
@@ -465,13 +475,54 @@ __device__ __forceinline__ void pairs(uint4 t, f2 (&p)[4]) {
     p[3] = pk2(bf16_lo(t.w), bf16_hi(t.w));
 }
 
-template <int NV, int VEC>
-__device__ __forceinline__ void unpack_acc(const f2 (&acc)[NV][VEC / 2], float (&o)[NV][VEC]) {
+// Row accumulator of one lane: NV vectors of VEC fp32 sums, either as packed
+// pairs updated with fma.rn.f32x2 or as plain floats updated with fmaf (the
+// same rounding per element).
+template <typename T, int NV, int VEC, bool PACKED> struct RowAcc;
+
+template <typename T, int NV, int VEC> struct RowAcc<T, NV, VEC, true> {
+    f2 a[NV][VEC / 2];
+    __device__ __forceinline__ void zero() {
 #pragma unroll
-    for (int k = 0; k < NV; ++k)
+        for (int k = 0; k < NV; ++k)
 #pragma unroll
-        for (int i = 0; i < VEC / 2; ++i) up2(acc[k][i], o[k][2 * i], o[k][2 * i + 1]);
-}
+            for (int i = 0; i < VEC / 2; ++i) a[k][i] = 0ull;
+    }
+    __device__ __forceinline__ void fma(int k, float w, typename Vec<T, VEC>::raw x) {
+        const f2 w2 = pk2(w, w);
+        f2 xp[VEC / 2];
+        pairs(x, xp);
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i) a[k][i] = ffma2(w2, xp[i], a[k][i]);
+    }
+    __device__ __forceinline__ void get(float (&o)[NV][VEC]) const {
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+#pragma unroll
+            for (int i = 0; i < VEC / 2; ++i) up2(a[k][i], o[k][2 * i], o[k][2 * i + 1]);
+    }
+};
+template <typename T, int NV, int VEC> struct RowAcc<T, NV, VEC, false> {
+    float a[NV][VEC];
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) a[k][v] = 0.f;
+    }
+    __device__ __forceinline__ void fma(int k, float w, typename Vec<T, VEC>::raw x) {
+        float xf[VEC];
+        Vec<T, VEC>::unpack(x, xf);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) a[k][v] = fmaf(w, xf[v], a[k][v]);
+    }
+    __device__ __forceinline__ void get(float (&o)[NV][VEC]) const {
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) o[k][v] = a[k][v];
+    }
+};
 
 // Same contract as k_tiles for 16-byte vectors (fp32 x 4, bf16 x 8) and a
 // single column tile, with the lane-group width G and the ring depth D fixed
@@ -509,9 +560,12 @@ k_tiles_ring(const Params P) {
     const unsigned gmask = (G == 32) ? FULL : (((1u << G) - 1u) << (lane & ~(G - 1)));
     const int H = int(P.H);
     const int HV = H / VEC;
+    // the ring path runs only for rows of exactly G x NV 16-byte vectors, so
+    // every lane's vectors are in range (constant-folded away)
     bool colok[NV];
 #pragma unroll
-    for (int k = 0; k < NV; ++k) colok[k] = gl + k * G < HV;
+    for (int k = 0; k < NV; ++k) colok[k] = true;
+    (void)HV;
 
     if (gid >= n_tiles_pad) {  // warps of empty rows: zeros
         const int64_t z = gid - n_tiles_pad;
@@ -564,27 +618,27 @@ k_tiles_ring(const Params P) {
     if (G + gl < len) { c_nxt = __ldcs(P.col + p0 + G + gl); e_nxt = __ldcs(P.order + p0 + G + gl); }
     if ((MODE & kSpmm) && gl < len) w_cur = load_w(P.w + e_cur);
 
+    const uint32_t row_bytes = uint32_t(H) * sizeof(T);
     auto issue = [&](int slot, int src) {
-        const T *Frow = F + int64_t(src) * H;
+        const char *Frow = reinterpret_cast<const char *>(F) + uint64_t(uint32_t(src)) * row_bytes;
 #pragma unroll
         for (int k = 0; k < NV; ++k)
-            if (colok[k]) cp_async16(my_s + uint32_t((slot * NV + k) * G * 16), Frow + k * G * VEC);
+            if (colok[k]) cp_async16(my_s + uint32_t((slot * NV + k) * G * 16), Frow + k * G * 16);
     };
+    constexpr int STEP = AG_RING_STEP;
+    static_assert(D % STEP == 0 && G % STEP == 0, "ring step");
 #pragma unroll
     for (int s = 0; s < D; ++s) {
         const int src = __shfl_sync(FULL, c_cur, s, G);
         if (s < len) issue(s, src);
-        cp_async_commit();
+        if (s % STEP == STEP - 1) cp_async_commit();
     }
 
-    f2 acc[NV][VEC / 2];
+    RowAcc<T, NV, VEC, AG_FFMA2 != 0> acc;
+    acc.zero();
     raw_t own[NV], own_next[NV];
 #pragma unroll
-    for (int k = 0; k < NV; ++k) {
-        own[k] = own_next[k] = Vec<T, VEC>::zero();
-#pragma unroll
-        for (int i = 0; i < VEC / 2; ++i) acc[k][i] = 0ull;
-    }
+    for (int k = 0; k < NV; ++k) own[k] = own_next[k] = Vec<T, VEC>::zero();
     if ((MODE & kSddmm) && active) {
         const T *Rrow = R + int64_t(row) * H;
         const T *Rnext = R + int64_t(__shfl_sync(gmask, la_row, 0, G)) * H;
@@ -599,7 +653,7 @@ k_tiles_ring(const Params P) {
 
     auto write_open_row = [&](float *slot) {
         float o[NV][VEC];
-        unpack_acc<NV, VEC>(acc, o);
+        acc.get(o);
         if (slot) store_slot<VEC, NV>(slot, 0, G, colok, o);
         else store_row<T, VEC, NV>(out + int64_t(row) * H, 0, G, colok, o);
     };
@@ -608,10 +662,7 @@ k_tiles_ring(const Params P) {
     auto next_row = [&]() {
         if ((MODE & kSpmm)) {
             write_open_row(before ? slot_head : nullptr);
-#pragma unroll
-            for (int q = 0; q < NV; ++q)
-#pragma unroll
-                for (int i = 0; i < VEC / 2; ++i) acc[q][i] = 0ull;
+            acc.zero();
         }
         before = false;
         row = __shfl_sync(gmask, la_row, la_k, G);
@@ -639,7 +690,6 @@ k_tiles_ring(const Params P) {
     // position p0 + base + j (valid: inside this group's tile); returns this
     // lane's part of the dot (kSddmm)
     auto consume = [&](int base, int j, bool valid) -> float {
-        cp_async_wait<D - 1>();
         const float wk = ((MODE & kSpmm)) ? __shfl_sync(FULL, w_cur, j, G) : 0.f;
         float d = 0.f;
         if (valid) {
@@ -649,15 +699,9 @@ k_tiles_ring(const Params P) {
             if (p0 + base + j == rend) next_row();
             // slots of out-of-range column vectors were never written: skip them
             if ((MODE & kSpmm)) {
-                const f2 w2 = pk2(wk, wk);
 #pragma unroll
-                for (int q = 0; q < NV; ++q) {
-                    if (!colok[q]) continue;
-                    f2 xp[VEC / 2];
-                    pairs(x[q], xp);
-#pragma unroll
-                    for (int i = 0; i < VEC / 2; ++i) acc[q][i] = ffma2(w2, xp[i], acc[q][i]);
-                }
+                for (int q = 0; q < NV; ++q)
+                    if (colok[q]) acc.fma(q, wk, x[q]);
             }
             if ((MODE & kSddmm)) {
 #pragma unroll
@@ -672,7 +716,7 @@ k_tiles_ring(const Params P) {
         const int src = (j + D < G) ? __shfl_sync(FULL, c_cur, (j + D) & (G - 1), G)
                                     : __shfl_sync(FULL, c_nxt, (j + D) & (G - 1), G);
         if (!check || base + j + D < len) issue(j % D, src);
-        cp_async_commit();
+        if (j % STEP == STEP - 1) cp_async_commit();
     };
 
     for (int base = 0; base < len_max; base += G) {
@@ -691,14 +735,18 @@ k_tiles_ring(const Params P) {
         if (base + G + D <= len_min) {
             float dots[G];
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                dots[j] = consume(base, j, true);
-                refill(base, j, false);
+            for (int j = 0; j < G; j += STEP) {
+                cp_async_wait<D / STEP - 1>();
+#pragma unroll
+                for (int t = 0; t < STEP; ++t) dots[j + t] = consume(base, j + t, true);
+#pragma unroll
+                for (int t = 0; t < STEP; ++t) refill(base, j + t, false);
             }
             if ((MODE & kSddmm)) P.dw[e_cur] = reduce_scatter<G>(dots, gl, FULL);
         } else {
 #pragma unroll 1
             for (int j = 0; j < G; ++j) {
+                if (j % STEP == 0) cp_async_wait<D / STEP - 1>();
                 float d = consume(base, j, base + j < len);
                 if ((MODE & kSddmm)) {
 #pragma unroll
@@ -735,9 +783,12 @@ k_dw_coo(const int32_t *__restrict__ src, const int32_t *__restrict__ dst, const
     const int64_t gid = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> LOG2G;
     const int gl = threadIdx.x & (G - 1);
     const int HV = H / VEC;
+    // the ring path runs only for rows of exactly G x NV 16-byte vectors, so
+    // every lane's vectors are in range (constant-folded away)
     bool colok[NV];
 #pragma unroll
-    for (int k = 0; k < NV; ++k) colok[k] = gl + k * G < HV;
+    for (int k = 0; k < NV; ++k) colok[k] = true;
+    (void)HV;
     // slot s: X piece k at my[((2s) * NV + k) * G], dY piece k at my[((2s + 1) * NV + k) * G]
     const uint4 *my = ring + (threadIdx.x >> LOG2G) * (2 * D * NV * G) + gl;
     const uint32_t my_s = smem_addr(my);
@@ -753,9 +804,10 @@ k_dw_coo(const int32_t *__restrict__ src, const int32_t *__restrict__ dst, const
     if (gl < len) { s_cur = __ldcs(src + p0 + gl); d_cur = __ldcs(dst + p0 + gl); }
     if (G + gl < len) { s_nxt = __ldcs(src + p0 + G + gl); d_nxt = __ldcs(dst + p0 + G + gl); }
 
+    const uint32_t row_bytes = uint32_t(H) * sizeof(T);
     auto issue = [&](int slot, int sv, int dv) {
-        const T *xr = X + int64_t(sv) * H;
-        const T *yr = dY + int64_t(dv) * H;
+        const T *xr = reinterpret_cast<const T *>(reinterpret_cast<const char *>(X) + uint64_t(uint32_t(sv)) * row_bytes);
+        const T *yr = reinterpret_cast<const T *>(reinterpret_cast<const char *>(dY) + uint64_t(uint32_t(dv)) * row_bytes);
 #pragma unroll
         for (int k = 0; k < NV; ++k)
             if (colok[k]) {
@@ -979,7 +1031,7 @@ void launch_main(const Params &P, const Shape &s, cudaStream_t st) {
     const int64_t groups = P.n_tiles + P.n_zero;
     const unsigned grid = unsigned((groups + groups_per_block - 1) / groups_per_block);
     if constexpr (sizeof(typename Vec<T, VEC>::raw) == 16 && NV <= 2) {
-        if (s.col_tiles == 1 && s.G >= 4) {
+        if (s.col_tiles == 1 && s.G >= 4 && int64_t(s.G) * NV * VEC == P.H) {
             switch (s.G) {
                 case 4: launch_ring<T, VEC, NV, 4, MODE>(P, st); return;
                 case 8: launch_ring<T, VEC, NV, 8, MODE>(P, st); return;
@@ -1111,9 +1163,141 @@ int check_call(const ag_graph *g, int64_t H, int dtype, const char *fn) {
     return AG_OK;
 }
 
+// Per-call scratch: [partial rows][weights, bucketed][weight gradient, bucketed]
+struct ScratchLayout {
+    size_t partial, w_b, dw_b, total;
+};
+ScratchLayout scratch_layout(const ag_graph *g, int64_t H) {
+    ScratchLayout L;
+    const bool spans = g->dir[0].n_span > 0 || g->dir[1].n_span > 0;
+    const size_t part = spans ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0;
+    const size_t ev = size_t(g->E) * 4;
+    L.partial = 0;
+    L.w_b = align_up(part);
+    L.dw_b = L.w_b + align_up(ev);
+    L.total = g->E > 0 ? L.dw_b + align_up(ev) : L.w_b;
+    return L;
+}
 size_t scratch_needed(const ag_graph *g, int64_t H) {
-    if (g->dir[0].n_span == 0 && g->dir[1].n_span == 0) return 0;
-    return size_t(2) * size_t(g->n_tiles) * size_t(H) * 4;
+    const ScratchLayout L = scratch_layout(g, H);
+    return (g->E > 0 || L.w_b > 0) ? L.total : 0;
+}
+
+// w_b[slot[e]] = w[e]: COO-ordered weights into the window-bucketed layout.
+// Reads are coalesced; the slots of consecutive ordinals that share a window
+// are consecutive, so the writes land in short runs that L2 merges.
+__global__ void k_bucket_scatter(const float *__restrict__ w, const int32_t *__restrict__ slot, int64_t E,
+                                 float *__restrict__ w_b) {
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x)
+        w_b[__ldcs(slot + e)] = __ldcs(w + e);
+}
+// dw[e] = dw_b[slot[e]]: the bucketed weight gradient back to COO order.
+__global__ void k_bucket_gather(const float *__restrict__ dw_b, const int32_t *__restrict__ slot, int64_t E,
+                                float *__restrict__ dw) {
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x)
+        __stcs(dw + e, dw_b[__ldcs(slot + e)]);
+}
+// Staged regrouping with the lowering's table: the ordinals of one chunk,
+// sorted by window, form runs of consecutive slots (slots of a window are
+// handed out in COO order), and slot + delta[window] is an ordinal's place in
+// that order.  TO_BUCKETS: w_b[slot[e]] = w[e] written run by run; otherwise
+// dw[e] = dw_b[slot[e]] read run by run.  Both sides coalesced, no atomics.
+constexpr int kStageItems = kStageChunk / kThreads;
+
+template <bool TO_BUCKETS>
+__global__ void __launch_bounds__(kThreads)
+k_bucket_staged(const float *__restrict__ in, const int32_t *__restrict__ slot,
+                const int32_t *__restrict__ delta_table, int64_t E, int shift, int nwin,
+                float *__restrict__ out) {
+    __shared__ int delta[kStageMaxWindows];
+    __shared__ int stage_slot[kStageChunk];
+    __shared__ float stage_val[kStageChunk];
+    const int64_t c0 = int64_t(blockIdx.x) * kStageChunk;
+    const int n = int(E - c0 < kStageChunk ? E - c0 : kStageChunk);
+    for (int b = threadIdx.x; b < nwin; b += kThreads) delta[b] = delta_table[int64_t(blockIdx.x) * nwin + b];
+    for (int i = threadIdx.x; i < n; i += kThreads) stage_slot[i] = -1;
+    __syncthreads();
+    // all global loads of the chunk first (independent), then the staging
+    int sl[kStageItems];
+    float v[kStageItems];
+#pragma unroll
+    for (int k = 0; k < kStageItems; ++k) {
+        const int i = k * kThreads + threadIdx.x;
+        sl[k] = i < n ? __ldcs(slot + c0 + i) : -1;
+        v[k] = (TO_BUCKETS && i < n) ? __ldcs(in + c0 + i) : 0.f;
+    }
+    int pos[kStageItems];
+#pragma unroll
+    for (int k = 0; k < kStageItems; ++k) {
+        pos[k] = -1;
+        if (sl[k] >= 0) {
+            const int p = sl[k] + delta[sl[k] >> shift];
+            if (p >= 0 && p < n) {  // always true for a consistent table
+                pos[k] = p;
+                stage_slot[p] = sl[k];
+                if (TO_BUCKETS) stage_val[p] = v[k];
+            }
+        }
+    }
+    __syncthreads();
+    // (every position of the chunk holds a slot in [0, E); the checks only
+    // keep an inconsistent table from turning into a stray access)
+    if (TO_BUCKETS) {
+#pragma unroll
+        for (int k = 0; k < kStageItems; ++k) {
+            const int i = k * kThreads + threadIdx.x;
+            const int s2 = i < n ? stage_slot[i] : -1;
+            if (s2 >= 0 && s2 < E) out[s2] = stage_val[i];
+        }
+    } else {
+        float g[kStageItems];
+#pragma unroll
+        for (int k = 0; k < kStageItems; ++k) {
+            const int i = k * kThreads + threadIdx.x;
+            const int s2 = i < n ? stage_slot[i] : -1;
+            g[k] = (s2 >= 0 && s2 < E) ? in[s2] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kStageItems; ++k) {
+            const int i = k * kThreads + threadIdx.x;
+            if (i < n) stage_val[i] = g[k];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kStageItems; ++k) {
+            const int i = k * kThreads + threadIdx.x;
+            if (i < n && pos[k] >= 0) __stcs(out + c0 + i, stage_val[pos[k]]);
+        }
+    }
+}
+
+// w_b[slot[e]] = w[e] (to_buckets) or dw[e] = dw_b[slot[e]]
+void regroup(bool to_buckets, const ag::Direction &D, const float *in, int64_t E, float *out, cudaStream_t st) {
+    if (AG_BUCKET_STAGED && D.stage_delta) {
+        const unsigned grid = unsigned(n_stage_chunks(E));
+        const int nwin = int(n_windows(E));
+        if (to_buckets)
+            k_bucket_staged<true><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, D.stage_delta, E, kWindowShift, nwin, out);
+        else
+            k_bucket_staged<false><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, D.stage_delta, E, kWindowShift, nwin, out);
+        return;
+    }
+    const int64_t b = (E + kThreads - 1) / kThreads;
+    const unsigned grid = unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
+    if (to_buckets) k_bucket_scatter<<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, E, out);
+    else k_bucket_gather<<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, E, out);
+}
+
+unsigned stream_grid(int64_t n) {
+    int64_t b = (n + kThreads - 1) / kThreads;
+    return unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
+}
+
+int check_scratch(const ag_graph *g, size_t need, const void *scratch, size_t scratch_bytes, const char *fn) {
+    if (need > 0 && (!scratch || scratch_bytes < need))
+        return fail(AG_ERR_WORKSPACE, "%s: scratch of %zu bytes, need %zu", fn, scratch_bytes, need);
+    if (!aligned(scratch, kAlign)) return fail(AG_ERR_WORKSPACE, "%s: scratch must be 256-byte aligned", fn);
+    return AG_OK;
 }
 
 // SpMM over direction d: out = A_w X (d = 0) or A_w^T dY (d = 1).
@@ -1123,10 +1307,9 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     if (rc != AG_OK) return rc;
     if (!F || !out || (g->E > 0 && !w)) return fail(AG_ERR_INVALID_ARG, "%s: null w, input or output", fn);
     const ag::Direction &D = g->dir[d];
-    const size_t need = D.n_span > 0 ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0;
-    if (need > 0 && (!scratch || scratch_bytes < need))
-        return fail(AG_ERR_WORKSPACE, "%s: scratch of %zu bytes, need %zu", fn, scratch_bytes, need);
-    if (!aligned(scratch, 16)) return fail(AG_ERR_WORKSPACE, "%s: scratch must be 16-byte aligned", fn);
+    const ScratchLayout SL = scratch_layout(g, H);
+    const size_t need = g->E > 0 ? SL.w_b + align_up(size_t(g->E) * 4) : SL.w_b;
+    if ((rc = check_scratch(g, need, scratch, scratch_bytes, fn)) != AG_OK) return rc;
     if (check_ptrs) {
         if ((rc = check_device_ptr(F, g->device, "input")) != AG_OK) return rc;
         if ((rc = check_device_ptr(out, g->device, "output")) != AG_OK) return rc;
@@ -1134,13 +1317,19 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
         if (need > 0 && (rc = check_device_ptr(scratch, g->device, "scratch")) != AG_OK) return rc;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *scr = static_cast<char *>(scratch);
     const Shape s = pick_shape(H, dtype, F, out, nullptr);
     Params P = base_params(g, D, H, s);
-    P.w = w;
     P.F = F;
     P.out = out;
-    P.partial = static_cast<float *>(scratch);
+    P.partial = reinterpret_cast<float *>(scr + SL.partial);
     P.n_zero = g->N - D.n_nz;
+    if (g->E > 0) {
+        float *w_b = reinterpret_cast<float *>(scr + SL.w_b);
+        regroup(true, D, w, g->E, w_b, st);
+        P.w = w_b;
+        P.order = D.bucket_of_pos;  // the kernels read w[order[p]]: here the bucketed slot
+    }
     if (P.n_tiles + P.n_zero > 0) dispatch_main<kSpmm>(P, s, dtype, st);
     if (D.n_span > 0) dispatch_fixup(D, P.partial, out, H, s, dtype, st);
     cudaError_t err = cudaGetLastError();
@@ -1148,35 +1337,44 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     return AG_OK;
 }
 
-// dw over the transpose CSR: owner = source row (X), gathered = dY[col_t].
-int sddmm(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, int dtype, void *stream,
-          const char *fn, bool check_ptrs) {
+// dw over the transpose CSR: owner = source row (X), gathered = dY[col_t];
+// each edge's dot goes to its bucketed slot, then back to COO order.
+int sddmm(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, int dtype, void *scratch,
+          size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs) {
     int rc = check_call(g, H, dtype, fn);
     if (rc != AG_OK) return rc;
     if (!X || !dY || (g->E > 0 && !dw)) return fail(AG_ERR_INVALID_ARG, "%s: null X, dY or dw", fn);
+    const ScratchLayout SL = scratch_layout(g, H);
+    const size_t need = g->E > 0 ? SL.total : 0;
+    if ((rc = check_scratch(g, need, scratch, scratch_bytes, fn)) != AG_OK) return rc;
     if (check_ptrs) {
         if ((rc = check_device_ptr(X, g->device, "X")) != AG_OK) return rc;
         if ((rc = check_device_ptr(dY, g->device, "dY")) != AG_OK) return rc;
         if (g->E > 0 && (rc = check_device_ptr(dw, g->device, "dw")) != AG_OK) return rc;
+        if (need > 0 && (rc = check_device_ptr(scratch, g->device, "scratch")) != AG_OK) return rc;
     }
     if (g->E == 0) return AG_OK;
     const ag::Direction &D = g->dir[1];
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape s = pick_shape(H, dtype, X, dY, nullptr);
 #if AG_DW_COO
-    if (s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8)) {
+    if (s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8) &&
+        int64_t(s.G) * s.nv * s.vec == H) {
         launch_dw_coo(g, X, dY, dw, H, dtype, s, st);
         cudaError_t err = cudaGetLastError();
         if (err != cudaSuccess) return cuda_fail(err, fn);
         return AG_OK;
     }
 #endif
+    float *dw_b = reinterpret_cast<float *>(static_cast<char *>(scratch) + SL.dw_b);
     Params P = base_params(g, D, H, s);
+    P.order = D.bucket_of_pos;
     P.F = dY;
     P.R = X;
-    P.dw = dw;
+    P.dw = dw_b;
     P.n_zero = 0;
     dispatch_main<kSddmm>(P, s, dtype, st);
+    regroup(false, D, dw_b, g->E, dw, st);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
@@ -1189,11 +1387,9 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
     if (rc != AG_OK) return rc;
     if (!X || !dY || !dX || (g->E > 0 && (!w || !dw)))
         return fail(AG_ERR_INVALID_ARG, "%s: null w, X, dY, dX or dw", fn);
-    const ag::Direction &D = g->dir[1];
-    const size_t need = D.n_span > 0 ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0;
-    if (need > 0 && (!scratch || scratch_bytes < need))
-        return fail(AG_ERR_WORKSPACE, "%s: scratch of %zu bytes, need %zu", fn, scratch_bytes, need);
-    if (!aligned(scratch, 16)) return fail(AG_ERR_WORKSPACE, "%s: scratch must be 16-byte aligned", fn);
+    const ScratchLayout SL = scratch_layout(g, H);
+    const size_t need = g->E > 0 ? SL.total : SL.w_b;
+    if ((rc = check_scratch(g, need, scratch, scratch_bytes, fn)) != AG_OK) return rc;
     if (check_ptrs) {
         if ((rc = check_device_ptr(X, g->device, "X")) != AG_OK) return rc;
         if ((rc = check_device_ptr(dY, g->device, "dY")) != AG_OK) return rc;
@@ -1202,28 +1398,32 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
         if (g->E > 0 && (rc = check_device_ptr(dw, g->device, "dw")) != AG_OK) return rc;
         if (need > 0 && (rc = check_device_ptr(scratch, g->device, "scratch")) != AG_OK) return rc;
     }
+    const ag::Direction &D = g->dir[1];
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape s = pick_shape(H, dtype, X, dY, dX);
-    const bool ring = s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8);
-    // The single walk scatters dw through transpose_order; that only pays when
-    // consecutive positions mostly share dw sectors (a source-sorted COO list).
-    // Otherwise the transpose-CSR SpMM and the COO-order SDDMM (coalesced dw)
-    // are faster.  Both choices give bitwise identical results.
-    const bool single_walk = ring && g->dw_locality >= kSingleWalkLocality;
-    if (!single_walk || g->E == 0) {
+    const bool ring = s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8) &&
+                      int64_t(s.G) * s.nv * s.vec == H;
+    if (!ring || g->E == 0) {
+        // shapes without the single walk: the two separate passes
         if ((rc = spmm(g, 1, w, dY, dX, H, dtype, scratch, scratch_bytes, stream, fn, false)) != AG_OK) return rc;
-        return sddmm(g, X, dY, dw, H, dtype, stream, fn, false);
+        return sddmm(g, X, dY, dw, H, dtype, scratch, scratch_bytes, stream, fn, false);
     }
+    char *scr = static_cast<char *>(scratch);
+    float *w_b = reinterpret_cast<float *>(scr + SL.w_b);
+    float *dw_b = reinterpret_cast<float *>(scr + SL.dw_b);
+    regroup(true, D, w, g->E, w_b, st);
     Params P = base_params(g, D, H, s);
-    P.w = w;
+    P.order = D.bucket_of_pos;
+    P.w = w_b;
     P.F = dY;
     P.R = X;
     P.out = dX;
-    P.dw = dw;
-    P.partial = static_cast<float *>(scratch);
+    P.dw = dw_b;
+    P.partial = reinterpret_cast<float *>(scr + SL.partial);
     P.n_zero = g->N - D.n_nz;
     dispatch_main<kBoth>(P, s, dtype, st);
     if (D.n_span > 0) dispatch_fixup(D, P.partial, dX, H, s, dtype, st);
+    regroup(false, D, dw_b, g->E, dw, st);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
@@ -1254,9 +1454,9 @@ int ag_spmm_dx(const ag_graph *g, const float *w, const void *dY, void *dX, int6
 }
 
 int ag_sddmm_dw(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, int dtype,
-                void *stream) {
+                void *scratch, size_t scratch_bytes, void *stream) {
     clear_error();
-    return sddmm(g, X, dY, dw, H, dtype, stream, "ag_sddmm_dw", true);
+    return sddmm(g, X, dY, dw, H, dtype, scratch, scratch_bytes, stream, "ag_sddmm_dw", true);
 }
 
 int ag_backward(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw, int64_t H,
@@ -1312,7 +1512,7 @@ int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, con
     auto copy = [&](void *to, const void *from, size_t n, cudaMemcpyKind k) {
         if (err == cudaSuccess && n > 0) err = cudaMemcpyAsync(to, from, n, k, st);
     };
-    const size_t scr = scratch_needed(g, H);
+    const size_t scr = scratch_needed(g, H);  // staging's scratch part
     copy(w, w_host, wb, cudaMemcpyHostToDevice);
     copy(X, X_host, feat, cudaMemcpyHostToDevice);
     if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy in");
@@ -1337,7 +1537,7 @@ int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, con
 // every GPU loading this library holds until the process exits.  In host code
 // the name g_static_scratch only stands in for the symbol; its device address
 // comes from cudaGetSymbolAddress below.
-static constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
+static constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
 
 namespace {
@@ -1369,7 +1569,8 @@ int ag_spmm_fwd_static_scratch(const ag_graph *g, const float *w, const void *X,
     clear_error();
     if (!g) return fail(AG_ERR_INVALID_ARG, "ag_spmm_fwd_static_scratch: null graph");
     if (H < 1) return fail(AG_ERR_SHAPE, "ag_spmm_fwd_static_scratch: H=%lld", (long long)H);
-    const size_t need = g->dir[0].n_span > 0 ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0;
+    const ScratchLayout SL = scratch_layout(g, H);
+    const size_t need = g->E > 0 ? SL.w_b + align_up(size_t(g->E) * 4) : SL.w_b;
     if (need > kStaticScratchBytes)
         return fail(AG_ERR_WORKSPACE,
                     "ag_spmm_fwd_static_scratch: this graph needs %zu bytes of scratch at H=%lld, more than the "

@@ -79,6 +79,9 @@ bool make_layout(int64_t N, int64_t E, Layout *L) {
         L->zero_rows[d] = take(n * 4);
         L->tile_nz[d] = take(tiles * 4);
         L->spans[d] = take((tiles < n ? tiles : n) * 16);  // a tile boundary cuts at most one row
+        L->bucket_a[d] = take(e * 4);
+        L->bucket_b[d] = take(e * 4);
+        L->stage_delta[d] = take(staged_regroup(E) ? size_t(n_stage_chunks(E) * n_windows(E)) * 4 : 0);
     }
     L->coo_src = take(e * 4);
     L->coo_dst = take(e * 4);

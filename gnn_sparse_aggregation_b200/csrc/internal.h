@@ -19,6 +19,20 @@ constexpr int kMaxTileEdges = 512;
 constexpr int kMinTileEdges = 32;
 constexpr int kFillGroups = 148 * 64;  // tiles wanted: SMs x resident lane groups
 constexpr int kLongSpanTiles = 8;
+// Weights (and the weight gradient) are regrouped per call into windows of
+// 2^kWindowShift consecutive CSR positions (4 MB of fp32), so that the
+// per-edge weight lookups of a tile stay inside one L2-resident window.
+#ifndef AG_WINDOW_SHIFT
+#define AG_WINDOW_SHIFT 20
+#endif
+constexpr int kWindowShift = AG_WINDOW_SHIFT;
+// The per-call regrouping passes move the weights of kStageChunk consecutive
+// COO ordinals at a time; stage_delta[c * windows + b] turns the slot of an
+// ordinal of chunk c in window b into its position in the chunk sorted by
+// window (slot + delta).  Built when the graph has at most kStageMaxWindows
+// windows.
+constexpr int kStageChunk = 4096;
+constexpr int kStageMaxWindows = 256;
 
 constexpr size_t kAlign = 256;
 
@@ -34,6 +48,12 @@ struct Direction {
     int32_t *zero_rows = nullptr;  // [N - n_nz] rows without edges, ascending
     int32_t *tile_nz = nullptr;    // [n_tiles] index into nz_rows of the row holding the tile's first position
     int4 *spans = nullptr;         // [n_span] {row, first tile, last tile, 0}: long spans first
+    // window-bucketed weight layout: bucket_of_coo[e] is the slot of COO
+    // ordinal e, bucket_of_pos[p] the slot read at CSR position p (slots of a
+    // window are that window's CSR positions, filled in COO order)
+    int32_t *bucket_of_coo = nullptr;  // [E]
+    int32_t *bucket_of_pos = nullptr;  // [E]
+    int32_t *stage_delta = nullptr;    // [chunks * windows] or null
     int64_t n_nz = 0, n_span = 0, n_span_long = 0, max_degree = 0;
 };
 
@@ -67,11 +87,15 @@ int check_device_ptr(const void *p, int device, const char *name);
 // Lowering-time workspace layout (shared by the size query and the lowering).
 struct Layout {
     size_t rowptr[2], col[2], order[2], nz_rows[2], nz_rowptr[2], zero_rows[2], tile_nz[2], spans[2];
+    size_t bucket_a[2], bucket_b[2], stage_delta[2];
     size_t coo_src, coo_dst;
     size_t keys_a, vals_a, keys_b, vals_b, hist, scan_tmp, aux, counters;
     size_t total;
 };
 bool make_layout(int64_t N, int64_t E, Layout *L);
+inline int64_t n_windows(int64_t E) { return E > 0 ? ((E - 1) >> kWindowShift) + 1 : 0; }
+inline int64_t n_stage_chunks(int64_t E) { return (E + kStageChunk - 1) / kStageChunk; }
+inline bool staged_regroup(int64_t E) { return E > 0 && n_windows(E) <= kStageMaxWindows; }
 int pick_tile_edges(int64_t E);
 inline int64_t n_tiles_for(int64_t E, int T) { return (E + T - 1) / T; }
 

@@ -19,6 +19,7 @@
 //      compacted (ids and first positions), the empty rows listed, the row
 //      holding the first position of every tile, and the rows cut by a tile
 //      boundary (long ones first).
+#include <climits>
 #include <cstdio>
 
 #include "internal.h"
@@ -296,6 +297,50 @@ __global__ void k_span_scatter(const int32_t *__restrict__ nz_rows, const int32_
     }
 }
 
+// out[order[p]] = p >> shift: the weight window of every COO ordinal.
+__global__ void k_window_keys(const int32_t *__restrict__ order, int64_t n, int shift, int32_t *__restrict__ out) {
+    for (int64_t p = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; p < n;
+         p += int64_t(gridDim.x) * blockDim.x)
+        out[order[p]] = int32_t(p >> shift);
+}
+
+// out[perm[i]] = i
+__global__ void k_invert(const int32_t *__restrict__ perm, int64_t n, int32_t *__restrict__ out) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x)
+        out[perm[i]] = int32_t(i);
+}
+
+// Per chunk of kStageChunk ordinals: for every window b that has ordinals in
+// the chunk, delta = (start of b's run in the chunk sorted by window) - (the
+// smallest slot of the chunk in b).  The slots of a window within a chunk are
+// consecutive, so slot + delta is the ordinal's position in the sorted chunk.
+__global__ void __launch_bounds__(256)
+k_stage_table(const int32_t *__restrict__ slot, int64_t E, int shift, int nwin, int32_t *__restrict__ delta) {
+    __shared__ int cnt[kStageMaxWindows];
+    __shared__ int first[kStageMaxWindows];
+    const int64_t c0 = int64_t(blockIdx.x) * kStageChunk;
+    const int n = int(E - c0 < kStageChunk ? E - c0 : kStageChunk);
+    for (int b = threadIdx.x; b < nwin; b += blockDim.x) {
+        cnt[b] = 0;
+        first[b] = INT_MAX;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int sl = slot[c0 + i];
+        atomicAdd(&cnt[sl >> shift], 1);
+        atomicMin(&first[sl >> shift], sl);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int b = 0; b < nwin; ++b) {
+            delta[int64_t(blockIdx.x) * nwin + b] = cnt[b] ? run - first[b] : 0;
+            run += cnt[b];
+        }
+    }
+}
+
 // Number of positions p > 0 whose ordinal lies in the same 8-ordinal
 // (32-byte) sector as the ordinal at p - 1.
 __global__ void k_sector_runs(const int32_t *__restrict__ order, int64_t n, unsigned long long *count) {
@@ -458,6 +503,23 @@ extern "C" int ag_graph_lower(const int32_t *src, const int32_t *dst, int64_t N,
         const int32_t *sorted = radix_sort(key, nullptr, E, key_bits, D.order, t, s);
         k_rowptr_search<<<grid_for(N + 1, 256), 256, 0, s>>>(sorted, E, N, D.rowptr);
         if (E > 0) k_gather<<<grid_for(E, 256), 256, 0, s>>>(D.order, other, E, D.col);
+
+        // window-bucketed weight layout (see kWindowShift): sort the COO
+        // ordinals stably by the window of their CSR position
+        if (E > 0) {
+            int32_t *A = I(L.bucket_a[d]), *B = I(L.bucket_b[d]);
+            k_window_keys<<<grid_for(E, 256), 256, 0, s>>>(D.order, E, kWindowShift, A);
+            radix_sort(A, nullptr, E, bit_length((E - 1) >> kWindowShift), B, t, s);  // B[slot] = ordinal
+            k_invert<<<grid_for(E, 256), 256, 0, s>>>(B, E, A);                        // A[ordinal] = slot
+            k_gather<<<grid_for(E, 256), 256, 0, s>>>(D.order, A, E, B);              // B[pos] = slot
+            D.bucket_of_coo = A;
+            D.bucket_of_pos = B;
+            if (staged_regroup(E)) {
+                D.stage_delta = I(L.stage_delta[d]);
+                k_stage_table<<<unsigned(n_stage_chunks(E)), 256, 0, s>>>(A, E, kWindowShift, int(n_windows(E)),
+                                                                         D.stage_delta);
+            }
+        }
 
         // 4. tile schedule
         err = cudaMemsetAsync(counters, 0, 8 * sizeof(int), s);

@@ -83,7 +83,7 @@ typedef struct ag_graph_stats {
     int64_t long_spanning_rows_f; /* of those, rows cut into more than 9 tiles */
     int64_t nonempty_rows_t, spanning_rows_t, long_spanning_rows_t; /* same, transpose CSR */
     size_t workspace_bytes_used;
-    double dw_locality;         /* share of transpose-CSR neighbours whose COO ordinals share a dw sector */
+    double dw_locality;         /* share of transpose-CSR neighbours whose COO ordinals share a 32-byte sector */
 } ag_graph_stats;
 
 /*
@@ -135,10 +135,13 @@ AG_API int ag_graph_arrays(const ag_graph *g, const int32_t **rowptr_f, const in
 AG_API int ag_graph_get_stats(const ag_graph *g, ag_graph_stats *out);
 
 /*
- * Device scratch, in bytes, that ag_spmm_fwd / ag_spmm_dx / ag_step_host need
- * for feature width H: two fp32 partial rows per tile for the rows that a
- * tile boundary cuts (2 x tiles x H x 4 bytes), 0 when no row is cut.  This
- * is O(E / tile_edges * H), never E x H.
+ * Device scratch, in bytes, that the per-call functions need for feature
+ * width H: two fp32 partial rows per tile for the rows that a tile boundary
+ * cuts (2 x tiles x H x 4 bytes, 0 when no row is cut), plus two float [E]
+ * buffers that hold the weights and the weight gradient regrouped by windows
+ * of 2^20 consecutive CSR positions (the weights stay in COO order in the
+ * caller's arrays; the regrouping keeps each tile's weight lookups inside
+ * one window).  O(E / tile_edges * H + E), never E x H.
  */
 AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
 
@@ -153,7 +156,7 @@ AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
  *   X        device [N, H] of dtype
  *   Y        device [N, H] of dtype, fully written; rows without in-edges are 0
  *   scratch  device buffer of ag_spmm_scratch_bytes(g, H) bytes (NULL if 0),
- *            16-byte aligned; its contents are scratch only
+ *            256-byte aligned; its contents are scratch only
  * Rows cut by tile boundaries are summed in fixed tile order, so results are
  * bitwise reproducible.  Errors: AG_ERR_INVALID_ARG, AG_ERR_SHAPE (H < 1 or N*H too
  * large), AG_ERR_DTYPE, AG_ERR_DEVICE, AG_ERR_WORKSPACE, AG_ERR_CUDA.
@@ -178,11 +181,12 @@ AG_API int ag_spmm_dx(const ag_graph *g, const float *w, const void *dY, void *d
  *
  *   X, dY    device [N, H] of dtype
  *   dw       device float [E], written in COO order (may be NULL when E == 0)
+ *   scratch  device buffer of ag_spmm_scratch_bytes(g, H) bytes (see there)
  * Every edge's value is computed independently (duplicates get equal values).
- * Errors as ag_spmm_fwd (no scratch is needed).
+ * Errors as ag_spmm_fwd.
  */
 AG_API int ag_sddmm_dw(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H,
-                int dtype, void *stream);
+                int dtype, void *scratch, size_t scratch_bytes, void *stream);
 
 /*
  * Feature gradient and weight gradient in one pass over the transpose CSR:
@@ -191,11 +195,7 @@ AG_API int ag_sddmm_dw(const ag_graph *g, const void *X, const void *dY, float *
  * experiment"); the fusion is this library's: every dY row gathered for an
  * edge feeds both the dX row of the edge's source and the edge's dot
  * product, so dY is gathered once for both gradients instead of twice.
- * Results are bitwise identical to ag_spmm_dx followed by ag_sddmm_dw.  The
- * single walk writes dw through transpose_order, which costs a 32-byte
- * sector per edge when the COO order is unrelated to the source order; so it
- * is used only when ag_graph_stats.dw_locality >= 0.5 (a source-sorted COO
- * list), and otherwise this call runs the two separate passes.
+ * Results are bitwise identical to ag_spmm_dx followed by ag_sddmm_dw.
  *
  *   w        device float [E], COO order
  *   X, dY    device [N, H] of dtype
@@ -236,9 +236,10 @@ AG_API int ag_step_host(const ag_graph *g, const float *w_host, const void *X_ho
  * device array built into the library instead of caller scratch.
  *
  *   - The built-in array holds ag_spmm_static_scratch_capacity() bytes
- *     (16 MiB) on every GPU that loads the library, until the process exits.
- *     A graph that needs more (2 x tiles x H x 4 bytes when a row is cut by
- *     a tile boundary) is rejected with AG_ERR_WORKSPACE; nothing is launched.
+ *     (32 MiB) on every GPU that loads the library, until the process exits.
+ *     A graph that needs more (the partial rows and the regrouped weights of
+ *     ag_spmm_scratch_bytes) is rejected with AG_ERR_WORKSPACE; nothing is
+ *     launched.
  *   - The call allocates nothing (no cudaMalloc, cudaFree or allocating
  *     library routine).  Its first call on a device looks up the array's
  *     device address there (cudaGetSymbolAddress); make that first call
@@ -247,7 +248,7 @@ AG_API int ag_step_host(const ag_graph *g, const float *w_host, const void *X_ho
  *   - All calls share the one array: calls whose work overlaps on the GPU
  *     (different streams, different host threads) race and must be ordered
  *     by the caller.  The array keeps the previous call's contents; no part
- *     of it has to start at zero, because every partial row a call reads is
+ *     of it has to start at zero, because everything a call reads from it is
  *     written earlier in the same call.
  * Arguments and other errors as ag_spmm_fwd.
  */

@@ -47,8 +47,7 @@ def test_matches_caller_scratch_forward_on_two_calls(case):
         H = 64 if "h64" in case else 256
         wl = workloads.custom(N, src, dst, H, seed=9, feature_dtype=dtype, device="cuda")
     g = agb.ag_graph_lower(wl.src, wl.dst, wl.N)
-    need = g.scratch_bytes(wl.H)
-    assert 0 < need <= agb.lib.ag_spmm_static_scratch_capacity()   # rows are cut by tiles
+    assert g.scratch_bytes(wl.H) > 0                        # this graph needs scratch
     ref = agb.ag_spmm_fwd(g, wl.w, wl.X)
     # elementwise scale of the tolerance: sum over in-edges of |w_e x|
     bound = agb.ag_spmm_fwd(g, wl.w.abs(), wl.X.abs()).double()
