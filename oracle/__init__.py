@@ -11,9 +11,15 @@ tinymesh "Weighted aggregation experiment" page ("Decision", "Edge order is
 explicit") and the COO loop of the PyTorch Geometric reading guide (Step 2,
 without the m x d temporary, which Step 3 says the fused path drops).
 
+The further aggregators (mean, GCN-normalised weights, edge-softmax
+attention) follow the same reading guide: Step 3 (GCN's normalised adjacency,
+the sum and mean reductions of spmm) and Step 4 (SDDMM scores, a softmax per
+destination row, then the SpMM).
+
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
-against the hand-derived "Exact witness" fixture, dense matrix products,
-library stable sorts, the adjoint identity and finite differences.
+and ``tests/test_oracle_ext_pins.py`` against the hand-derived "Exact
+witness" fixture, dense matrix products, library stable sorts and softmax,
+closed forms, the adjoint identity and finite differences.
 """
 from __future__ import annotations
 
@@ -55,8 +61,16 @@ def _load():
         lib.oracle_spmm_rows.argtypes = [_I64, _I64, _I64, _P, _P, _P, _P, ctypes.c_int,
                                          _I64, _P, _P, _P]
         lib.oracle_dw_edges.argtypes = [_I64, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _P]
+        for name in ("oracle_mean_fwd", "oracle_mean_dx", "oracle_mean_dw"):
+            getattr(lib, name).argtypes = [_I64, _I64, _I64, _P, _P, _P, _P, _P, _P]
+        lib.oracle_gcn_norm.argtypes = [_I64, _I64, _P, _P, _P, _P]
+        lib.oracle_attn_fwd.argtypes = [_I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_double,
+                                        _P, _P, _P, _P]
+        lib.oracle_attn_bwd.argtypes = [_I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_double,
+                                        _P, _P, _P, _P, _P, _P]
         for name in ("oracle_lower", "oracle_fwd", "oracle_dx", "oracle_dw",
-                     "oracle_spmm_rows", "oracle_dw_edges"):
+                     "oracle_spmm_rows", "oracle_dw_edges", "oracle_mean_fwd", "oracle_mean_dx",
+                     "oracle_mean_dw", "oracle_gcn_norm", "oracle_attn_fwd", "oracle_attn_bwd"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -171,3 +185,75 @@ def dw_edges(src, dst, N: int, X, dY, edges, with_bound: bool = False):
                                    edges.shape[0], _ptr(edges), _ptr(out),
                                    _ptr(bound) if with_bound else None))
     return (out, bound) if with_bound else out
+
+
+# ----------------------------------------------------------------------------- further aggregators
+
+def mean_fwd(src, dst, N: int, w, X, with_bound: bool = False):
+    """Y[r] = sum over edges into r of w_e X[src_e], divided by the number of
+    edges into r (0 for rows without edges); fp64 [N, H]."""
+    return _spmm_like("oracle_mean_fwd", src, dst, N, w, X, N, with_bound)
+
+
+def mean_dx(src, dst, N: int, w, dY, with_bound: bool = False):
+    """dX[s] = sum over edges out of s of (w_e / cnt(dst_e)) dY[dst_e]."""
+    return _spmm_like("oracle_mean_dx", src, dst, N, w, dY, N, with_bound)
+
+
+def mean_dw(src, dst, N: int, X, dY, with_bound: bool = False):
+    """dw_e = dot(X[src_e], dY[dst_e]) / cnt(dst_e), COO order."""
+    src, dst = _i32(src), _i32(dst)
+    X, dY = _f32(X), _f32(dY)
+    E = src.shape[0]
+    out = np.zeros(E, np.float64)
+    bound = np.zeros(E, np.float64) if with_bound else None
+    _check(_load().oracle_mean_dw(N, E, X.shape[1], _ptr(src), _ptr(dst), _ptr(X), _ptr(dY),
+                                  _ptr(out), _ptr(bound) if with_bound else None))
+    return (out, bound) if with_bound else out
+
+
+def gcn_norm(src, dst, N: int, w=None) -> np.ndarray:
+    """D^-1/2 A_w D^-1/2 as edge weights (COO order), D = weighted in-degree;
+    w=None means unit weights; deg <= 0 contributes a factor 0."""
+    src, dst = _i32(src), _i32(dst)
+    E = src.shape[0]
+    wf = None if w is None else _f32(w)
+    out = np.zeros(E, np.float64)
+    _check(_load().oracle_gcn_norm(N, E, _ptr(src), _ptr(dst), None if wf is None else _ptr(wf),
+                                   _ptr(out)))
+    return out
+
+
+def attn_fwd(src, dst, N: int, Q, K, V, scale: float, with_bound: bool = False):
+    """Edge-softmax attention: returns (s, alpha, Y[, bound]) with s and alpha
+    in COO order (fp64) and Y [N, H] (fp64)."""
+    src, dst = _i32(src), _i32(dst)
+    Q, K, V = _f32(Q), _f32(K), _f32(V)
+    E = src.shape[0]
+    H = Q.shape[1]
+    s = np.zeros(E, np.float64)
+    alpha = np.zeros(E, np.float64)
+    Y = np.zeros((N, H), np.float64)
+    bound = np.zeros_like(Y) if with_bound else None
+    _check(_load().oracle_attn_fwd(N, E, H, _ptr(src), _ptr(dst), _ptr(Q), _ptr(K), _ptr(V),
+                                   float(scale), _ptr(s), _ptr(alpha), _ptr(Y),
+                                   _ptr(bound) if with_bound else None))
+    return (s, alpha, Y, bound) if with_bound else (s, alpha, Y)
+
+
+def attn_bwd(src, dst, N: int, Q, K, V, scale: float, alpha, dY):
+    """Gradients (dQ, dK, dV, ds) of the attention for upstream gradient dY;
+    alpha is the fp64 alpha of attn_fwd."""
+    src, dst = _i32(src), _i32(dst)
+    Q, K, V, dY = _f32(Q), _f32(K), _f32(V), _f32(dY)
+    alpha = np.ascontiguousarray(np.asarray(alpha, np.float64))
+    E = src.shape[0]
+    H = Q.shape[1]
+    dQ = np.zeros((N, H), np.float64)
+    dK = np.zeros((N, H), np.float64)
+    dV = np.zeros((N, H), np.float64)
+    ds = np.zeros(E, np.float64)
+    _check(_load().oracle_attn_bwd(N, E, H, _ptr(src), _ptr(dst), _ptr(Q), _ptr(K), _ptr(V),
+                                   float(scale), _ptr(alpha), _ptr(dY), _ptr(dQ), _ptr(dK),
+                                   _ptr(dV), _ptr(ds)))
+    return dQ, dK, dV, ds

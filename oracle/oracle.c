@@ -280,3 +280,232 @@ int oracle_dw_edges(int64_t N, int64_t E, int64_t H, const int32_t *src,
     }
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------
+ * Further aggregators over the same adjacency (PyTorch Geometric reading
+ * guide: Step 3 "the fused path" for the degree-normalised GCN weights and
+ * the sum-or-mean reductions of spmm, "Done when" on reduce='max'; Step 4
+ * "SDDMM: the second primitive, forced by attention" for the edge softmax).
+ * ------------------------------------------------------------------------ */
+
+/* number of edges into every destination; NULL when out of memory */
+static double *in_counts(int64_t N, int64_t E, const int32_t *dst)
+{
+    double *cnt = (double *)calloc((size_t)N, sizeof(double));
+    if (!cnt)
+        return NULL;
+    for (int64_t e = 0; e < E; ++e)
+        cnt[dst[e]] += 1.0;
+    return cnt;
+}
+
+/*
+ * Mean aggregation: Y[r, h] = (sum over edges e into r of w_e X[src_e, h]) / cnt(r),
+ * cnt(r) = number of edges into r (duplicates counted); rows with no edge are 0.
+ * absb receives the same sums of |w_e X[src_e, h]| / cnt(r).
+ */
+int oracle_mean_fwd(int64_t N, int64_t E, int64_t H, const int32_t *src, const int32_t *dst,
+                    const float *w, const float *X, double *Y, double *absb)
+{
+    int rc = oracle_fwd(N, E, H, src, dst, w, X, Y, absb);
+    if (rc)
+        return rc;
+    double *cnt = in_counts(N, E, dst);
+    if (!cnt)
+        return ORACLE_NO_MEMORY;
+    for (int64_t r = 0; r < N; ++r) {
+        if (cnt[r] == 0.0)
+            continue;
+        for (int64_t h = 0; h < H; ++h) {
+            Y[r * H + h] /= cnt[r];
+            if (absb)
+                absb[r * H + h] /= cnt[r];
+        }
+    }
+    free(cnt);
+    return ORACLE_OK;
+}
+
+/*
+ * Gradients of the mean aggregation for an upstream gradient dY:
+ *   dX[src_e, h] += (w_e / cnt(dst_e)) dY[dst_e, h]
+ *   dw_e = dot(X[src_e], dY[dst_e]) / cnt(dst_e)
+ */
+int oracle_mean_dx(int64_t N, int64_t E, int64_t H, const int32_t *src, const int32_t *dst,
+                   const float *w, const float *dY, double *dX, double *absb)
+{
+    if (!sizes_ok(N, E) || H < 1)
+        return ORACLE_BAD_SIZE;
+    if (!indices_ok(N, E, src, dst))
+        return ORACLE_BAD_INDEX;
+    double *cnt = in_counts(N, E, dst);
+    if (!cnt)
+        return ORACLE_NO_MEMORY;
+    memset(dX, 0, (size_t)(N * H) * sizeof(double));
+    if (absb)
+        memset(absb, 0, (size_t)(N * H) * sizeof(double));
+    for (int64_t e = 0; e < E; ++e) {
+        double a = (double)w[e] / cnt[dst[e]];
+        const float *gd = dY + (int64_t)dst[e] * H;
+        double *xs = dX + (int64_t)src[e] * H;
+        for (int64_t h = 0; h < H; ++h) {
+            xs[h] += a * (double)gd[h];
+            if (absb)
+                absb[(int64_t)src[e] * H + h] += fabs(a * (double)gd[h]);
+        }
+    }
+    free(cnt);
+    return ORACLE_OK;
+}
+
+int oracle_mean_dw(int64_t N, int64_t E, int64_t H, const int32_t *src, const int32_t *dst,
+                   const float *X, const float *dY, double *dw, double *absb)
+{
+    int rc = oracle_dw(N, E, H, src, dst, X, dY, dw, absb);
+    if (rc)
+        return rc;
+    double *cnt = in_counts(N, E, dst);
+    if (!cnt)
+        return ORACLE_NO_MEMORY;
+    for (int64_t e = 0; e < E; ++e) {
+        dw[e] /= cnt[dst[e]];
+        if (absb)
+            absb[e] /= cnt[dst[e]];
+    }
+    free(cnt);
+    return ORACLE_OK;
+}
+
+/*
+ * GCN normalisation of the weights, D^-1/2 A_w D^-1/2:
+ *   deg(i) = sum of w_e over the edges into i (w = NULL: every w_e = 1),
+ *   out_e  = w_e / sqrt(deg(src_e)) / sqrt(deg(dst_e)),
+ * with deg^-1/2 taken as 0 where deg(i) <= 0 (no normalisation is defined
+ * there).  Self-loops are part of the edge list given.
+ */
+int oracle_gcn_norm(int64_t N, int64_t E, const int32_t *src, const int32_t *dst,
+                    const float *w, double *out)
+{
+    if (!sizes_ok(N, E))
+        return ORACLE_BAD_SIZE;
+    if (!indices_ok(N, E, src, dst))
+        return ORACLE_BAD_INDEX;
+    double *deg = (double *)calloc((size_t)N, sizeof(double));
+    if (!deg)
+        return ORACLE_NO_MEMORY;
+    for (int64_t e = 0; e < E; ++e)
+        deg[dst[e]] += w ? (double)w[e] : 1.0;
+    for (int64_t i = 0; i < N; ++i)
+        deg[i] = deg[i] > 0.0 ? 1.0 / sqrt(deg[i]) : 0.0;
+    for (int64_t e = 0; e < E; ++e)
+        out[e] = deg[src[e]] * (w ? (double)w[e] : 1.0) * deg[dst[e]];
+    free(deg);
+    return ORACLE_OK;
+}
+
+/*
+ * Edge-softmax attention over the forward adjacency (SDDMM scores, a softmax
+ * per destination row, then the SpMM with the normalised scores):
+ *   s_e     = scale * dot(Q[dst_e], K[src_e])
+ *   m_r     = max of s_e over the edges into r
+ *   alpha_e = exp(s_e - m_r) / (sum over edges e' into r of exp(s_e' - m_r))
+ *   Y[r, h] = sum over edges e into r of alpha_e V[src_e, h]
+ * Rows without edges have Y = 0.  s and alpha are written in COO order;
+ * absb[r, h] = sum over the same edges of |alpha_e V[src_e, h]|.
+ */
+int oracle_attn_fwd(int64_t N, int64_t E, int64_t H, const int32_t *src, const int32_t *dst,
+                    const float *Q, const float *K, const float *V, double scale,
+                    double *s, double *alpha, double *Y, double *absb)
+{
+    if (!sizes_ok(N, E) || H < 1)
+        return ORACLE_BAD_SIZE;
+    if (!indices_ok(N, E, src, dst))
+        return ORACLE_BAD_INDEX;
+    double *m = (double *)malloc((size_t)N * sizeof(double));
+    double *z = (double *)calloc((size_t)N, sizeof(double));
+    if (!m || !z) {
+        free(m);
+        free(z);
+        return ORACLE_NO_MEMORY;
+    }
+    for (int64_t r = 0; r < N; ++r)
+        m[r] = -INFINITY;
+    for (int64_t e = 0; e < E; ++e) {
+        const float *q = Q + (int64_t)dst[e] * H;
+        const float *k = K + (int64_t)src[e] * H;
+        double acc = 0.0;
+        for (int64_t h = 0; h < H; ++h)
+            acc += (double)q[h] * (double)k[h];
+        s[e] = scale * acc;
+        if (s[e] > m[dst[e]])
+            m[dst[e]] = s[e];
+    }
+    for (int64_t e = 0; e < E; ++e)
+        z[dst[e]] += exp(s[e] - m[dst[e]]);
+    for (int64_t e = 0; e < E; ++e)
+        alpha[e] = exp(s[e] - m[dst[e]]) / z[dst[e]];
+    memset(Y, 0, (size_t)(N * H) * sizeof(double));
+    if (absb)
+        memset(absb, 0, (size_t)(N * H) * sizeof(double));
+    for (int64_t e = 0; e < E; ++e) {
+        const float *v = V + (int64_t)src[e] * H;
+        double *y = Y + (int64_t)dst[e] * H;
+        for (int64_t h = 0; h < H; ++h) {
+            y[h] += alpha[e] * (double)v[h];
+            if (absb)
+                absb[(int64_t)dst[e] * H + h] += fabs(alpha[e] * (double)v[h]);
+        }
+    }
+    free(m);
+    free(z);
+    return ORACLE_OK;
+}
+
+/*
+ * Gradients of the attention for an upstream gradient dY (alpha as computed
+ * by oracle_attn_fwd), from the chain rule through the row softmax:
+ *   dalpha_e = dot(dY[dst_e], V[src_e])
+ *   c_r      = sum over edges e into r of alpha_e dalpha_e
+ *   ds_e     = alpha_e (dalpha_e - c_{dst_e})
+ *   dQ[r]    = scale * sum over edges e into r   of ds_e K[src_e]
+ *   dK[s]    = scale * sum over edges e out of s of ds_e Q[dst_e]
+ *   dV[s]    =         sum over edges e out of s of alpha_e dY[dst_e]
+ * ds (COO order) is returned too.
+ */
+int oracle_attn_bwd(int64_t N, int64_t E, int64_t H, const int32_t *src, const int32_t *dst,
+                    const float *Q, const float *K, const float *V, double scale,
+                    const double *alpha, const float *dY,
+                    double *dQ, double *dK, double *dV, double *ds)
+{
+    if (!sizes_ok(N, E) || H < 1)
+        return ORACLE_BAD_SIZE;
+    if (!indices_ok(N, E, src, dst))
+        return ORACLE_BAD_INDEX;
+    double *c = (double *)calloc((size_t)N, sizeof(double));
+    if (!c)
+        return ORACLE_NO_MEMORY;
+    for (int64_t e = 0; e < E; ++e) {
+        const float *g = dY + (int64_t)dst[e] * H;
+        const float *v = V + (int64_t)src[e] * H;
+        double acc = 0.0;
+        for (int64_t h = 0; h < H; ++h)
+            acc += (double)g[h] * (double)v[h];
+        ds[e] = acc;  /* dalpha_e for now */
+        c[dst[e]] += alpha[e] * acc;
+    }
+    for (int64_t e = 0; e < E; ++e)
+        ds[e] = alpha[e] * (ds[e] - c[dst[e]]);
+    memset(dQ, 0, (size_t)(N * H) * sizeof(double));
+    memset(dK, 0, (size_t)(N * H) * sizeof(double));
+    memset(dV, 0, (size_t)(N * H) * sizeof(double));
+    for (int64_t e = 0; e < E; ++e) {
+        const int64_t r = dst[e], so = src[e];
+        for (int64_t h = 0; h < H; ++h) {
+            dQ[r * H + h] += scale * ds[e] * (double)K[so * H + h];
+            dK[so * H + h] += scale * ds[e] * (double)Q[r * H + h];
+            dV[so * H + h] += alpha[e] * (double)dY[r * H + h];
+        }
+    }
+    free(c);
+    return ORACLE_OK;
+}
