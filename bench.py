@@ -81,6 +81,18 @@ def algorithmic_bytes(N, E, H, elem):
     return {"fwd": spmm, "dx": spmm, "dw": dw, "backward": backward}
 
 
+def launches_per_step_of(st, wl):
+    """Kernels one step launches: ag_spmm_fwd = weight regroup + tile walk
+    (+ fixup when rows span tiles); ag_backward on the single-walk shapes (the
+    whole width in one lane group pass, as for H=128) = weight regroup + fused
+    walk (+ fixup) + dw regroup back to COO order."""
+    if wl.E == 0:
+        return int(wl.N > 0) * 2
+    fwd = 2 + int(st["spanning_rows_f"] > 0)
+    bwd = 3 + int(st["spanning_rows_t"] > 0)
+    return fwd + bwd
+
+
 def source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gnn_sparse_aggregation_b200", "csrc")
@@ -89,6 +101,10 @@ def source_hash():
             with open(os.path.join(csrc, fn), "rb") as f:
                 h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
+
+
+def traffic_key(args):
+    return args.workload if args.rmat_scale is None else f"{args.workload}@scale{args.rmat_scale}"
 
 
 def ncu_traffic(workload, kernel_op):
@@ -386,7 +402,7 @@ def our_arm(args):
         gbs = algo[op] / (avg[op] / 1e3) / 1e9
         kernels[op] = {"ms": avg[op], "EH_per_s": wl.E * wl.H / (avg[op] / 1e3),
                        "algorithmic_bytes": algo[op], "GB_per_s": gbs, "frac_of_peak": gbs / hbm}
-    launches_per_step = (1 + (st["spanning_rows_f"] > 0)) + (1 + (st["spanning_rows_t"] > 0))
+    launches_per_step = launches_per_step_of(st, wl)
     line = {
         "metric": METRIC,
         "value": whole_job_rate(world, wl.E * wl.H, K, ms),
@@ -400,7 +416,7 @@ def our_arm(args):
                      "peak": hbm, "unit": "GB/s",
                      "frac": algo[dominant] / (avg[dominant] / 1e3) / 1e9 / hbm,
                      "peak_source": f"{peak_kind} hbm_gbs",
-                     "traffic": ncu_traffic(args.workload, dominant)},
+                     "traffic": ncu_traffic(traffic_key(args), dominant)},
         "kernels": kernels,
         "lowering_ms": lower_ms[1], "lowering_first_call_ms": lower_ms[0],
         "schedule": {k: st[k] for k in ("tile_edges", "tiles", "spanning_rows_f", "long_spanning_rows_f",

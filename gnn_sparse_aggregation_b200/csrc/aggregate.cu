@@ -696,7 +696,8 @@ k_tiles_ring(const Params P) {
             raw_t x[NV];
 #pragma unroll
             for (int q = 0; q < NV; ++q) x[q] = *reinterpret_cast<const raw_t *>(my + ((j % D) * NV + q) * G);
-            if (p0 + base + j == rend) next_row();
+            // row ends are rare next to edges: keep the edge path straight-line
+            if (__builtin_expect(p0 + base + j == rend, 0)) next_row();
             // slots of out-of-range column vectors were never written: skip them
             if ((MODE & kSpmm)) {
 #pragma unroll
