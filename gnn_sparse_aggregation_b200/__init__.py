@@ -25,7 +25,7 @@ import re
 import torch
 
 __all__ = ["AggraphError", "Graph", "ag_graph_lower", "ag_spmm_fwd", "ag_spmm_dx", "ag_sddmm_dw", "ag_backward",
-           "ag_step_host", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
+           "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_step_host", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
            "declared_symbols", "AG_F32", "AG_BF16"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaggraph.so")
@@ -78,6 +78,11 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_spmm_dx.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_sddmm_dw.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_mean_fwd.argtypes = [_P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_mean_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_gcn_norm_scratch_bytes.argtypes = [_P]
+    handle.ag_gcn_norm_scratch_bytes.restype = _SZ
+    handle.ag_gcn_norm.argtypes = [_P, _P, _P, _P, _SZ, _P]
     handle.ag_spmm_fwd_static_scratch.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
     handle.ag_spmm_static_scratch_capacity.argtypes = []
     handle.ag_spmm_static_scratch_capacity.restype = _SZ
@@ -90,7 +95,8 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_status_string.argtypes = [_I]
     handle.ag_status_string.restype = ctypes.c_char_p
     for name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
-                 "ag_sddmm_dw", "ag_backward", "ag_spmm_fwd_static_scratch", "ag_step_host", "ag_abi_version"):
+                 "ag_sddmm_dw", "ag_backward", "ag_spmm_fwd_static_scratch", "ag_step_host", "ag_abi_version",
+                 "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm"):
         getattr(handle, name).restype = _I
     return handle
 
@@ -244,8 +250,9 @@ def _check_edge_vec(g: Graph, name: str, t: torch.Tensor) -> None:
         raise AggraphError(2, f"{name} must be [E={g.E}], got {tuple(t.shape)}")
 
 
-def _spmm(fn, g: Graph, w, F, out, stream, names):
-    _check_edge_vec(g, "w", w)
+def _spmm(fn, g: Graph, w, F, out, stream, names, w_optional=False):
+    if w is not None or not w_optional:
+        _check_edge_vec(g, "w", w)
     code = _check_feat(g, names[0], F)
     H = F.shape[1]
     if out is None:
@@ -307,6 +314,53 @@ def ag_backward(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, dX
     _check(lib.ag_backward(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(dX), _ptr(dw), H, code, _ptr(scr),
                            0 if scr is None else scr.numel(), _stream(g.device, stream)))
     return dX, dw
+
+
+def ag_mean_fwd(g: Graph, w, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """Y[r] = mean over the edges into r of w_e X[src_e] (w=None: unit weights)."""
+    return _spmm(lib.ag_mean_fwd, g, w, X, out, stream, ("X", "Y"), w_optional=True)
+
+
+def ag_mean_backward(g: Graph, w, X: torch.Tensor, dY: torch.Tensor, dX=None, dw=None, want_dw=True,
+                     stream=None):
+    """Gradients of ag_mean_fwd: (dX, dw) with dw = None when want_dw is False."""
+    if w is not None:
+        _check_edge_vec(g, "w", w)
+    code = _check_feat(g, "X", X)
+    if _check_feat(g, "dY", dY) != code or dY.shape != X.shape:
+        raise AggraphError(2, "X and dY must have the same shape and dtype")
+    if dX is None:
+        dX = torch.empty_like(dY)
+    elif dX.shape != dY.shape or dX.dtype != dY.dtype:
+        raise AggraphError(2, "dX must match dY in shape and dtype")
+    else:
+        _need_cuda("dX", dX)
+    if want_dw:
+        if dw is None:
+            dw = torch.empty(g.E, dtype=torch.float32, device=g.device)
+        else:
+            _check_edge_vec(g, "dw", dw)
+    else:
+        dw = None
+    H = X.shape[1]
+    scr = g.scratch(H)
+    _check(lib.ag_mean_backward(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(dX), _ptr(dw), H, code, _ptr(scr),
+                                0 if scr is None else scr.numel(), _stream(g.device, stream)))
+    return dX, dw
+
+
+def ag_gcn_norm(g: Graph, w=None, out=None, stream=None) -> torch.Tensor:
+    """GCN-normalised weights D^-1/2 A_w D^-1/2 in COO order (w=None: unit weights)."""
+    if w is not None:
+        _check_edge_vec(g, "w", w)
+    if out is None:
+        out = torch.empty(g.E, dtype=torch.float32, device=g.device)
+    else:
+        _check_edge_vec(g, "w_norm", out)
+    n = int(lib.ag_gcn_norm_scratch_bytes(g.handle))
+    scr = torch.empty(max(n, 1), dtype=torch.uint8, device=g.device)
+    _check(lib.ag_gcn_norm(g.handle, _ptr(w), _ptr(out), _ptr(scr), n, _stream(g.device, stream)))
+    return out
 
 
 def ag_spmm_fwd_static_scratch(g: Graph, w: torch.Tensor, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:

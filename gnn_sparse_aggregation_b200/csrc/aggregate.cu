@@ -39,17 +39,14 @@ namespace {
 #define AG_W_STREAM 0     // 1: weight lookups loaded evict-first; 0: normal caching (the bucketed
                           // weights of a window are reused from L2 by the window's tiles)
 #endif
-#ifndef AG_DW_COO
-#define AG_DW_COO 0       // 1: standalone weight gradient walks COO order (two gathers per edge)
-#endif
-#ifndef AG_FFMA2
-#define AG_FFMA2 0        // 1: packed fp32x2 FMAs in the ring SpMM (0: scalar fmaf, fewer register moves)
-#endif
 #ifndef AG_RING_STEP
 #define AG_RING_STEP 1    // positions per cp.async wait/commit in the ring SpMM (1 or 2)
 #endif
 #ifndef AG_BUCKET_STAGED
 #define AG_BUCKET_STAGED 1  // 1: weight regrouping passes stage a chunk in shared memory (coalesced)
+#endif
+#ifndef AG_CHUNK
+#define AG_CHUNK 8        // positions per unrolled chunk of a gradient-walk batch (the rest is rolled)
 #endif
 #ifndef AG_MAX_LANES
 #define AG_MAX_LANES 16   // lanes that share one row (fewer lanes: more 16-byte vectors per lane)
@@ -59,6 +56,7 @@ constexpr int kThreads = 256;
 constexpr int kUnroll = 4;     // gathered rows in flight per lane (register path)
 constexpr int kMinBlocks = 4;  // resident CTAs per SM the register path is compiled for
 constexpr int kRingDepth = AG_RING_DEPTH;
+constexpr int kChunk = AG_CHUNK;
 
 enum Mode { kSpmm = 1, kSddmm = 2, kBoth = 3 };  // kBoth: feature and weight gradient in one walk
 
@@ -425,6 +423,36 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[G], int gl, unsigned 
     return v[0];
 }
 
+// Positions per unrolled chunk of a ring batch of G with depth D: the largest
+// power of two <= min(kChunk, G) that divides G - D, so that a chunk never
+// straddles the switch from this batch's column indices to the next batch's.
+constexpr int chunk_of(int G, int D) {
+    int u = kChunk < G ? kChunk : G;
+    while (u > 1 && u < G && (G - D) % u != 0) u >>= 1;
+    return u;
+}
+
+// The same for a chunk of U <= G items spread over G lanes: U - 1 halving
+// exchanges leave lane l with item (l mod U) summed over its U-lane block,
+// then log2(G / U) butterfly steps add the blocks, so that every lane l holds
+// the total of item (l mod U).  For U == G this is reduce_scatter<G>.
+template <int U, int G>
+__device__ __forceinline__ float reduce_chunk(float (&v)[U], int gl, unsigned gmask) {
+#pragma unroll
+    for (int s = U / 2; s >= 1; s >>= 1) {
+        const bool upper = gl & s;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+            const float send = upper ? v[i] : v[i + s];
+            const float keep = upper ? v[i + s] : v[i];
+            v[i] = keep + __shfl_xor_sync(gmask, send, s, G);
+        }
+    }
+#pragma unroll
+    for (int o = U; o < G; o <<= 1) v[0] += __shfl_xor_sync(gmask, v[0], o, G);
+    return v[0];
+}
+
 // dot product of two raw 16-byte vectors, accumulated in order into c.
 // bf16: fma.rn.f32.bf16 multiplies two bf16 values exactly and adds in fp32
 // with one rounding -- the same result as widening both to fp32 first.
@@ -452,57 +480,10 @@ __device__ __forceinline__ float dot_raw(uint4 a, uint4 b, float c) {
     return dot2_bf16(a.w, b.w, c);
 }
 
-// Packed fp32 pairs (Blackwell FFMA2): fma.rn.f32x2 rounds each half exactly
-// like fma.rn.f32, so a pair update equals two scalar fmaf calls.
-using f2 = unsigned long long;
-__device__ __forceinline__ f2 pk2(float a, float b) {
-    f2 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void up2(f2 r, float &a, float &b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
-__device__ __forceinline__ f2 ffma2(f2 a, f2 b, f2 c) {
-    f2 d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-// a raw 16-byte vector as fp32 pairs, in element order
-__device__ __forceinline__ void pairs(float4 t, f2 (&p)[2]) { p[0] = pk2(t.x, t.y); p[1] = pk2(t.z, t.w); }
-__device__ __forceinline__ void pairs(uint4 t, f2 (&p)[4]) {
-    p[0] = pk2(bf16_lo(t.x), bf16_hi(t.x));
-    p[1] = pk2(bf16_lo(t.y), bf16_hi(t.y));
-    p[2] = pk2(bf16_lo(t.z), bf16_hi(t.z));
-    p[3] = pk2(bf16_lo(t.w), bf16_hi(t.w));
-}
-
-// Row accumulator of one lane: NV vectors of VEC fp32 sums, either as packed
-// pairs updated with fma.rn.f32x2 or as plain floats updated with fmaf (the
-// same rounding per element).
-template <typename T, int NV, int VEC, bool PACKED> struct RowAcc;
-
-template <typename T, int NV, int VEC> struct RowAcc<T, NV, VEC, true> {
-    f2 a[NV][VEC / 2];
-    __device__ __forceinline__ void zero() {
-#pragma unroll
-        for (int k = 0; k < NV; ++k)
-#pragma unroll
-            for (int i = 0; i < VEC / 2; ++i) a[k][i] = 0ull;
-    }
-    __device__ __forceinline__ void fma(int k, float w, typename Vec<T, VEC>::raw x) {
-        const f2 w2 = pk2(w, w);
-        f2 xp[VEC / 2];
-        pairs(x, xp);
-#pragma unroll
-        for (int i = 0; i < VEC / 2; ++i) a[k][i] = ffma2(w2, xp[i], a[k][i]);
-    }
-    __device__ __forceinline__ void get(float (&o)[NV][VEC]) const {
-#pragma unroll
-        for (int k = 0; k < NV; ++k)
-#pragma unroll
-            for (int i = 0; i < VEC / 2; ++i) up2(a[k][i], o[k][2 * i], o[k][2 * i + 1]);
-    }
-};
-template <typename T, int NV, int VEC> struct RowAcc<T, NV, VEC, false> {
+// Row accumulator of one lane: NV vectors of VEC fp32 sums updated with
+// fmaf.  (Packed fma.rn.f32x2 pairs round the same way per element but cost
+// register moves to form the pairs; measured slower here.)
+template <typename T, int NV, int VEC> struct RowAcc {
     float a[NV][VEC];
     __device__ __forceinline__ void zero() {
 #pragma unroll
@@ -634,7 +615,7 @@ k_tiles_ring(const Params P) {
         if (s % STEP == STEP - 1) cp_async_commit();
     }
 
-    RowAcc<T, NV, VEC, AG_FFMA2 != 0> acc;
+    RowAcc<T, NV, VEC> acc;
     acc.zero();
     raw_t own[NV], own_next[NV];
 #pragma unroll
@@ -687,15 +668,15 @@ k_tiles_ring(const Params P) {
             }
         }
     };
-    // position p0 + base + j (valid: inside this group's tile); returns this
-    // lane's part of the dot (kSddmm)
-    auto consume = [&](int base, int j, bool valid) -> float {
+    // position p0 + base + j, held in ring slot `slot` (valid: inside this
+    // group's tile); returns this lane's part of the dot (kSddmm)
+    auto consume = [&](int base, int j, int slot, bool valid) -> float {
         const float wk = ((MODE & kSpmm)) ? __shfl_sync(FULL, w_cur, j, G) : 0.f;
         float d = 0.f;
         if (valid) {
             raw_t x[NV];
 #pragma unroll
-            for (int q = 0; q < NV; ++q) x[q] = *reinterpret_cast<const raw_t *>(my + ((j % D) * NV + q) * G);
+            for (int q = 0; q < NV; ++q) x[q] = *reinterpret_cast<const raw_t *>(my + (slot * NV + q) * G);
             // row ends are rare next to edges: keep the edge path straight-line
             if (__builtin_expect(p0 + base + j == rend, 0)) next_row();
             // slots of out-of-range column vectors were never written: skip them
@@ -712,13 +693,19 @@ k_tiles_ring(const Params P) {
         }
         return d;
     };
-    // refill slot j % D with position base + j + D (this batch or the next)
-    auto refill = [&](int base, int j, bool check) {
-        const int src = (j + D < G) ? __shfl_sync(FULL, c_cur, (j + D) & (G - 1), G)
-                                    : __shfl_sync(FULL, c_nxt, (j + D) & (G - 1), G);
-        if (!check || base + j + D < len) issue(j % D, src);
+    // refill `slot` (= j mod D) with position base + j + D, whose column
+    // index lane (j + D) mod G holds in `cols` (c_cur: this batch, c_nxt: the next)
+    auto refill = [&](int base, int j, int slot, int cols, bool check) {
+        const int src = __shfl_sync(FULL, cols, (j + D) & (G - 1), G);
+        if (!check || base + j + D < len) issue(slot, src);
         if (j % STEP == STEP - 1) cp_async_commit();
     };
+    // the unguarded batch of the gradient walks runs in chunks of U positions
+    // (rolled), so that their longer row-switch code is inlined U times rather
+    // than G times; the forward walk keeps the whole batch unrolled
+    constexpr int U = MODE == kSpmm ? G : chunk_of(G, D);
+    static_assert(U % STEP == 0 && (U == G || (G - D) % U == 0) && (U >= D ? U % D == 0 : D % U == 0),
+                  "chunk shape");
 
     for (int base = 0; base < len_max; base += G) {
         if (base > 0) {
@@ -734,27 +721,39 @@ k_tiles_ring(const Params P) {
             e_nn = __ldcs(P.order + p0 + base + 2 * G + gl);
         }
         if (base + G + D <= len_min) {
-            float dots[G];
+#pragma unroll 1
+            for (int c = 0; c < G / U; ++c) {
+                float dots[U];
+                const int j0 = U == G ? 0 : c * U;
+                const int slot0 = U >= D ? 0 : j0 % D;
 #pragma unroll
-            for (int j = 0; j < G; j += STEP) {
-                cp_async_wait<D / STEP - 1>();
+                for (int t = 0; t < U; t += STEP) {
+                    cp_async_wait<D / STEP - 1>();
 #pragma unroll
-                for (int t = 0; t < STEP; ++t) dots[j + t] = consume(base, j + t, true);
+                    for (int u = 0; u < STEP; ++u)
+                        dots[t + u] = consume(base, j0 + t + u, U >= D ? (t + u) % D : slot0 + t + u, true);
+                    // (G - D) is a multiple of U: one source batch per chunk
 #pragma unroll
-                for (int t = 0; t < STEP; ++t) refill(base, j + t, false);
+                    for (int u = 0; u < STEP; ++u)
+                        refill(base, j0 + t + u, U >= D ? (t + u) % D : slot0 + t + u,
+                               (U == G ? t + u + D < G : j0 + D < G) ? c_cur : c_nxt, false);
+                }
+                if ((MODE & kSddmm)) {
+                    const float d = reduce_chunk<U, G>(dots, gl, FULL);
+                    if ((gl & ~(U - 1)) == j0) P.dw[e_cur] = d;  // lane j0 + t: position j0 + t
+                }
             }
-            if ((MODE & kSddmm)) P.dw[e_cur] = reduce_scatter<G>(dots, gl, FULL);
         } else {
 #pragma unroll 1
             for (int j = 0; j < G; ++j) {
                 if (j % STEP == 0) cp_async_wait<D / STEP - 1>();
-                float d = consume(base, j, base + j < len);
+                float d = consume(base, j, j % D, base + j < len);
                 if ((MODE & kSddmm)) {
 #pragma unroll
                     for (int o = G / 2; o > 0; o >>= 1) d += __shfl_xor_sync(FULL, d, o, G);
                     if (gl == j && base + j < len) P.dw[e_cur] = d;
                 }
-                refill(base, j, true);
+                refill(base, j, j % D, j + D < G ? c_cur : c_nxt, true);
             }
         }
     }
@@ -762,116 +761,6 @@ k_tiles_ring(const Params P) {
         if (before) write_open_row(slot_head);
         else if (rend > p0 + len) write_open_row(slot_tail);
         else write_open_row(nullptr);
-    }
-    cp_async_wait<0>();
-}
-
-// Weight gradient in COO order: lane group per tile of T consecutive COO
-// ordinals; both endpoint rows (X[src_e], dY[dst_e]) travel through the
-// shared-memory ring, and after the batch reduce-scatter lane j writes dw of
-// the batch's ordinal j, so the dw stores are coalesced.  The per-lane
-// partial dots and the reduction tree are those of the CSR walk, so both
-// walks give bitwise identical dw.
-template <typename T, int VEC, int NV, int G, int D>
-__global__ void __launch_bounds__(kThreads)
-k_dw_coo(const int32_t *__restrict__ src, const int32_t *__restrict__ dst, const void *Xv, const void *dYv,
-         float *__restrict__ dw, int E, int H, int T_tile, int64_t n_tiles) {
-    using raw_t = typename Vec<T, VEC>::raw;
-    static_assert(sizeof(raw_t) == 16 && G >= D && G % D == 0, "ring layout");
-    constexpr unsigned FULL = 0xffffffffu;
-    extern __shared__ uint4 ring[];
-    constexpr int LOG2G = G == 32 ? 5 : G == 16 ? 4 : G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
-    const int64_t gid = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> LOG2G;
-    const int gl = threadIdx.x & (G - 1);
-    const int HV = H / VEC;
-    // the ring path runs only for rows of exactly G x NV 16-byte vectors, so
-    // every lane's vectors are in range (constant-folded away)
-    bool colok[NV];
-#pragma unroll
-    for (int k = 0; k < NV; ++k) colok[k] = true;
-    (void)HV;
-    // slot s: X piece k at my[((2s) * NV + k) * G], dY piece k at my[((2s + 1) * NV + k) * G]
-    const uint4 *my = ring + (threadIdx.x >> LOG2G) * (2 * D * NV * G) + gl;
-    const uint32_t my_s = smem_addr(my);
-    const bool active = gid < n_tiles;
-    const int p0 = active ? int(gid) * T_tile : 0;
-    const int len = active ? min(T_tile, E - p0) : 0;
-    const int len_max = __reduce_max_sync(FULL, len);
-    const int len_min = __reduce_min_sync(FULL, len);
-    const T *X = static_cast<const T *>(Xv) + gl * VEC;
-    const T *dY = static_cast<const T *>(dYv) + gl * VEC;
-
-    int s_cur = 0, d_cur = 0, s_nxt = 0, d_nxt = 0, s_nn = 0, d_nn = 0;
-    if (gl < len) { s_cur = __ldcs(src + p0 + gl); d_cur = __ldcs(dst + p0 + gl); }
-    if (G + gl < len) { s_nxt = __ldcs(src + p0 + G + gl); d_nxt = __ldcs(dst + p0 + G + gl); }
-
-    const uint32_t row_bytes = uint32_t(H) * sizeof(T);
-    auto issue = [&](int slot, int sv, int dv) {
-        const T *xr = reinterpret_cast<const T *>(reinterpret_cast<const char *>(X) + uint64_t(uint32_t(sv)) * row_bytes);
-        const T *yr = reinterpret_cast<const T *>(reinterpret_cast<const char *>(dY) + uint64_t(uint32_t(dv)) * row_bytes);
-#pragma unroll
-        for (int k = 0; k < NV; ++k)
-            if (colok[k]) {
-                cp_async16(my_s + uint32_t(((2 * slot) * NV + k) * G * 16), xr + k * G * VEC);
-                cp_async16(my_s + uint32_t(((2 * slot + 1) * NV + k) * G * 16), yr + k * G * VEC);
-            }
-    };
-#pragma unroll
-    for (int q = 0; q < D; ++q) {
-        const int sv = __shfl_sync(FULL, s_cur, q, G), dv = __shfl_sync(FULL, d_cur, q, G);
-        if (q < len) issue(q, sv, dv);
-        cp_async_commit();
-    }
-    auto consume = [&](int j, bool valid) -> float {
-        cp_async_wait<D - 1>();
-        float d = 0.f;
-        if (valid) {
-#pragma unroll
-            for (int q = 0; q < NV; ++q)
-                if (colok[q]) {
-                    const raw_t a = *reinterpret_cast<const raw_t *>(my + ((2 * (j % D)) * NV + q) * G);
-                    const raw_t b = *reinterpret_cast<const raw_t *>(my + ((2 * (j % D) + 1) * NV + q) * G);
-                    d = dot_raw(a, b, d);
-                }
-        }
-        return d;
-    };
-    auto refill = [&](int base, int j, bool check) {
-        const int lanej = (j + D) & (G - 1);
-        const int sv = (j + D < G) ? __shfl_sync(FULL, s_cur, lanej, G) : __shfl_sync(FULL, s_nxt, lanej, G);
-        const int dv = (j + D < G) ? __shfl_sync(FULL, d_cur, lanej, G) : __shfl_sync(FULL, d_nxt, lanej, G);
-        if (!check || base + j + D < len) issue(j % D, sv, dv);
-        cp_async_commit();
-    };
-    for (int base = 0; base < len_max; base += G) {
-        if (base > 0) {
-            s_cur = s_nxt; d_cur = d_nxt;
-            s_nxt = s_nn; d_nxt = d_nn;
-        }
-        s_nn = 0;
-        d_nn = 0;
-        if (base + 2 * G + gl < len) {
-            s_nn = __ldcs(src + p0 + base + 2 * G + gl);
-            d_nn = __ldcs(dst + p0 + base + 2 * G + gl);
-        }
-        if (base + G + D <= len_min) {
-            float dots[G];
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-                dots[j] = consume(j, true);
-                refill(base, j, false);
-            }
-            __stcs(dw + p0 + base + gl, reduce_scatter<G>(dots, gl, FULL));
-        } else {
-#pragma unroll 1
-            for (int j = 0; j < G; ++j) {
-                float d = consume(j, base + j < len);
-#pragma unroll
-                for (int o = G / 2; o > 0; o >>= 1) d += __shfl_xor_sync(FULL, d, o, G);
-                if (gl == j && base + j < len) dw[p0 + base + j] = d;
-                refill(base, j, true);
-            }
-        }
     }
     cp_async_wait<0>();
 }
@@ -1099,44 +988,6 @@ void dispatch_fixup(const ag::Direction &D, const float *partial, void *out, int
     }
 }
 
-template <typename T, int VEC, int NV, int G>
-void launch_dw_coo_g(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, cudaStream_t st) {
-    constexpr int D = kRingDepth < G ? kRingDepth : G;
-    const size_t smem = size_t(kThreads) * 2 * D * NV * 16;
-    static bool configured = false;
-    if (!configured) {
-        cudaFuncSetAttribute(k_dw_coo<T, VEC, NV, G, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        configured = true;
-    }
-    const int64_t per_warp = 32 / G;
-    const int64_t groups = (g->n_tiles + per_warp - 1) / per_warp * per_warp;
-    const unsigned grid = unsigned((groups + kThreads / G - 1) / (kThreads / G));
-    k_dw_coo<T, VEC, NV, G, D><<<grid, kThreads, smem, st>>>(g->coo_src, g->coo_dst, X, dY, dw, int(g->E), int(H),
-                                                            g->tile_edges, g->n_tiles);
-}
-
-template <typename T, int VEC, int NV>
-void launch_dw_coo_nv(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, const Shape &s,
-                      cudaStream_t st) {
-    switch (s.G) {
-        case 4: launch_dw_coo_g<T, VEC, NV, 4>(g, X, dY, dw, H, st); break;
-        case 8: launch_dw_coo_g<T, VEC, NV, 8>(g, X, dY, dw, H, st); break;
-        case 16: launch_dw_coo_g<T, VEC, NV, 16>(g, X, dY, dw, H, st); break;
-        default: launch_dw_coo_g<T, VEC, NV, 32>(g, X, dY, dw, H, st); break;
-    }
-}
-
-void launch_dw_coo(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, int dtype,
-                   const Shape &s, cudaStream_t st) {
-    if (dtype == AG_F32) {
-        if (s.nv == 1) launch_dw_coo_nv<float, 4, 1>(g, X, dY, dw, H, s, st);
-        else launch_dw_coo_nv<float, 4, 2>(g, X, dY, dw, H, s, st);
-    } else {
-        if (s.nv == 1) launch_dw_coo_nv<bf16_t, 8, 1>(g, X, dY, dw, H, s, st);
-        else launch_dw_coo_nv<bf16_t, 8, 2>(g, X, dY, dw, H, s, st);
-    }
-}
-
 Params base_params(const ag_graph *g, const ag::Direction &D, int64_t H, const Shape &s) {
     Params P{};
     P.col = D.col;
@@ -1184,19 +1035,40 @@ size_t scratch_needed(const ag_graph *g, int64_t H) {
     return (g->E > 0 || L.w_b > 0) ? L.total : 0;
 }
 
-// w_b[slot[e]] = w[e]: COO-ordered weights into the window-bucketed layout.
-// Reads are coalesced; the slots of consecutive ordinals that share a window
-// are consecutive, so the writes land in short runs that L2 merges.
+// Optional per-edge factor applied while regrouping: divide the value of COO
+// edge e by the in-degree of its destination (mean aggregation).  dst = null:
+// no factor.
+struct EdgeScale {
+    const int32_t *dst = nullptr;     // COO destinations [E]
+    const int32_t *rowptr = nullptr;  // forward CSR row pointers [N + 1]
+};
+__device__ __forceinline__ float per_dst(float v, const EdgeScale &sc, int64_t e) {
+    const int d = __ldcs(sc.dst + e);
+    return __fdiv_rn(v, float(sc.rowptr[d + 1] - sc.rowptr[d]));  // >= 1: the edge itself
+}
+
+// w_b[slot[e]] = w[e] (w = null: 1): COO-ordered weights into the
+// window-bucketed layout.  Reads are coalesced; the slots of consecutive
+// ordinals that share a window are consecutive, so the writes land in short
+// runs that L2 merges.
+template <bool SCALED>
 __global__ void k_bucket_scatter(const float *__restrict__ w, const int32_t *__restrict__ slot, int64_t E,
-                                 float *__restrict__ w_b) {
-    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x)
-        w_b[__ldcs(slot + e)] = __ldcs(w + e);
+                                 EdgeScale sc, float *__restrict__ w_b) {
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
+        float v = w ? __ldcs(w + e) : 1.f;
+        if (SCALED) v = per_dst(v, sc, e);
+        w_b[__ldcs(slot + e)] = v;
+    }
 }
 // dw[e] = dw_b[slot[e]]: the bucketed weight gradient back to COO order.
+template <bool SCALED>
 __global__ void k_bucket_gather(const float *__restrict__ dw_b, const int32_t *__restrict__ slot, int64_t E,
-                                float *__restrict__ dw) {
-    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x)
-        __stcs(dw + e, dw_b[__ldcs(slot + e)]);
+                                EdgeScale sc, float *__restrict__ dw) {
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
+        float v = dw_b[__ldcs(slot + e)];
+        if (SCALED) v = per_dst(v, sc, e);
+        __stcs(dw + e, v);
+    }
 }
 // Staged regrouping with the lowering's table: the ordinals of one chunk,
 // sorted by window, form runs of consecutive slots (slots of a window are
@@ -1205,10 +1077,10 @@ __global__ void k_bucket_gather(const float *__restrict__ dw_b, const int32_t *_
 // dw[e] = dw_b[slot[e]] read run by run.  Both sides coalesced, no atomics.
 constexpr int kStageItems = kStageChunk / kThreads;
 
-template <bool TO_BUCKETS>
+template <bool TO_BUCKETS, bool SCALED>
 __global__ void __launch_bounds__(kThreads)
 k_bucket_staged(const float *__restrict__ in, const int32_t *__restrict__ slot,
-                const int32_t *__restrict__ delta_table, int64_t E, int shift, int nwin,
+                const int32_t *__restrict__ delta_table, int64_t E, int shift, int nwin, EdgeScale sc,
                 float *__restrict__ out) {
     __shared__ int delta[kStageMaxWindows];
     __shared__ int stage_slot[kStageChunk];
@@ -1225,7 +1097,8 @@ k_bucket_staged(const float *__restrict__ in, const int32_t *__restrict__ slot,
     for (int k = 0; k < kStageItems; ++k) {
         const int i = k * kThreads + threadIdx.x;
         sl[k] = i < n ? __ldcs(slot + c0 + i) : -1;
-        v[k] = (TO_BUCKETS && i < n) ? __ldcs(in + c0 + i) : 0.f;
+        v[k] = (TO_BUCKETS && i < n) ? (in ? __ldcs(in + c0 + i) : 1.f) : 0.f;
+        if (TO_BUCKETS && SCALED && i < n) v[k] = per_dst(v[k], sc, c0 + i);
     }
     int pos[kStageItems];
 #pragma unroll
@@ -1267,31 +1140,37 @@ k_bucket_staged(const float *__restrict__ in, const int32_t *__restrict__ slot,
 #pragma unroll
         for (int k = 0; k < kStageItems; ++k) {
             const int i = k * kThreads + threadIdx.x;
-            if (i < n && pos[k] >= 0) __stcs(out + c0 + i, stage_val[pos[k]]);
+            if (i < n && pos[k] >= 0)
+                __stcs(out + c0 + i, SCALED ? per_dst(stage_val[pos[k]], sc, c0 + i) : stage_val[pos[k]]);
         }
     }
 }
 
-// w_b[slot[e]] = w[e] (to_buckets) or dw[e] = dw_b[slot[e]]
-void regroup(bool to_buckets, const ag::Direction &D, const float *in, int64_t E, float *out, cudaStream_t st) {
+template <bool SCALED>
+void regroup_as(bool to_buckets, const ag::Direction &D, const float *in, int64_t E, const EdgeScale &sc,
+                float *out, cudaStream_t st) {
     if (AG_BUCKET_STAGED && D.stage_delta) {
         const unsigned grid = unsigned(n_stage_chunks(E));
         const int nwin = int(n_windows(E));
         if (to_buckets)
-            k_bucket_staged<true><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, D.stage_delta, E, kWindowShift, nwin, out);
+            k_bucket_staged<true, SCALED><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, D.stage_delta, E,
+                                                                      kWindowShift, nwin, sc, out);
         else
-            k_bucket_staged<false><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, D.stage_delta, E, kWindowShift, nwin, out);
+            k_bucket_staged<false, SCALED><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, D.stage_delta, E,
+                                                                       kWindowShift, nwin, sc, out);
         return;
     }
     const int64_t b = (E + kThreads - 1) / kThreads;
     const unsigned grid = unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
-    if (to_buckets) k_bucket_scatter<<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, E, out);
-    else k_bucket_gather<<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, E, out);
+    if (to_buckets) k_bucket_scatter<SCALED><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, E, sc, out);
+    else k_bucket_gather<SCALED><<<grid, kThreads, 0, st>>>(in, D.bucket_of_coo, E, sc, out);
 }
-
-unsigned stream_grid(int64_t n) {
-    int64_t b = (n + kThreads - 1) / kThreads;
-    return unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
+// w_b[slot[e]] = w[e] (to_buckets; w = null: 1) or dw[e] = dw_b[slot[e]],
+// each divided by the in-degree of e's destination when sc.dst is set
+void regroup(bool to_buckets, const ag::Direction &D, const float *in, int64_t E, float *out, cudaStream_t st,
+             const EdgeScale &sc = EdgeScale{}) {
+    if (sc.dst) regroup_as<true>(to_buckets, D, in, E, sc, out, st);
+    else regroup_as<false>(to_buckets, D, in, E, sc, out, st);
 }
 
 int check_scratch(const ag_graph *g, size_t need, const void *scratch, size_t scratch_bytes, const char *fn) {
@@ -1302,11 +1181,22 @@ int check_scratch(const ag_graph *g, size_t need, const void *scratch, size_t sc
 }
 
 // SpMM over direction d: out = A_w X (d = 0) or A_w^T dY (d = 1).
+EdgeScale mean_scale(const ag_graph *g, bool mean) {
+    EdgeScale sc;
+    if (mean) {
+        sc.dst = g->coo_dst;
+        sc.rowptr = g->dir[0].rowptr;
+    }
+    return sc;
+}
+
+// mean: divide every edge by the in-degree of its destination (w may then be
+// null for unit weights).
 int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int64_t H, int dtype,
-         void *scratch, size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs) {
+         void *scratch, size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs, bool mean = false) {
     int rc = check_call(g, H, dtype, fn);
     if (rc != AG_OK) return rc;
-    if (!F || !out || (g->E > 0 && !w)) return fail(AG_ERR_INVALID_ARG, "%s: null w, input or output", fn);
+    if (!F || !out || (g->E > 0 && !w && !mean)) return fail(AG_ERR_INVALID_ARG, "%s: null w, input or output", fn);
     const ag::Direction &D = g->dir[d];
     const ScratchLayout SL = scratch_layout(g, H);
     const size_t need = g->E > 0 ? SL.w_b + align_up(size_t(g->E) * 4) : SL.w_b;
@@ -1314,7 +1204,7 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     if (check_ptrs) {
         if ((rc = check_device_ptr(F, g->device, "input")) != AG_OK) return rc;
         if ((rc = check_device_ptr(out, g->device, "output")) != AG_OK) return rc;
-        if (g->E > 0 && (rc = check_device_ptr(w, g->device, "w")) != AG_OK) return rc;
+        if (g->E > 0 && w && (rc = check_device_ptr(w, g->device, "w")) != AG_OK) return rc;
         if (need > 0 && (rc = check_device_ptr(scratch, g->device, "scratch")) != AG_OK) return rc;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1327,7 +1217,7 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     P.n_zero = g->N - D.n_nz;
     if (g->E > 0) {
         float *w_b = reinterpret_cast<float *>(scr + SL.w_b);
-        regroup(true, D, w, g->E, w_b, st);
+        regroup(true, D, w, g->E, w_b, st, mean_scale(g, mean));
         P.w = w_b;
         P.order = D.bucket_of_pos;  // the kernels read w[order[p]]: here the bucketed slot
     }
@@ -1341,7 +1231,7 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
 // dw over the transpose CSR: owner = source row (X), gathered = dY[col_t];
 // each edge's dot goes to its bucketed slot, then back to COO order.
 int sddmm(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H, int dtype, void *scratch,
-          size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs) {
+          size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs, bool mean = false) {
     int rc = check_call(g, H, dtype, fn);
     if (rc != AG_OK) return rc;
     if (!X || !dY || (g->E > 0 && !dw)) return fail(AG_ERR_INVALID_ARG, "%s: null X, dY or dw", fn);
@@ -1358,15 +1248,6 @@ int sddmm(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H
     const ag::Direction &D = g->dir[1];
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape s = pick_shape(H, dtype, X, dY, nullptr);
-#if AG_DW_COO
-    if (s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8) &&
-        int64_t(s.G) * s.nv * s.vec == H) {
-        launch_dw_coo(g, X, dY, dw, H, dtype, s, st);
-        cudaError_t err = cudaGetLastError();
-        if (err != cudaSuccess) return cuda_fail(err, fn);
-        return AG_OK;
-    }
-#endif
     float *dw_b = reinterpret_cast<float *>(static_cast<char *>(scratch) + SL.dw_b);
     Params P = base_params(g, D, H, s);
     P.order = D.bucket_of_pos;
@@ -1375,19 +1256,23 @@ int sddmm(const ag_graph *g, const void *X, const void *dY, float *dw, int64_t H
     P.dw = dw_b;
     P.n_zero = 0;
     dispatch_main<kSddmm>(P, s, dtype, st);
-    regroup(false, D, dw_b, g->E, dw, st);
+    regroup(false, D, dw_b, g->E, dw, st, mean_scale(g, mean));
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
 }
 
 // Feature gradient and weight gradient in one walk of the transpose CSR.
+// mean: the gradients of the mean aggregation (w may be null for unit
+// weights, dw null when no weight gradient is wanted).
 int backward(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw, int64_t H,
-             int dtype, void *scratch, size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs) {
+             int dtype, void *scratch, size_t scratch_bytes, void *stream, const char *fn, bool check_ptrs,
+             bool mean = false) {
     int rc = check_call(g, H, dtype, fn);
     if (rc != AG_OK) return rc;
-    if (!X || !dY || !dX || (g->E > 0 && (!w || !dw)))
+    if (!X || !dY || !dX || (g->E > 0 && (!w || !dw) && !mean))
         return fail(AG_ERR_INVALID_ARG, "%s: null w, X, dY, dX or dw", fn);
+    if (mean && !dw) return spmm(g, 1, w, dY, dX, H, dtype, scratch, scratch_bytes, stream, fn, check_ptrs, true);
     const ScratchLayout SL = scratch_layout(g, H);
     const size_t need = g->E > 0 ? SL.total : SL.w_b;
     if ((rc = check_scratch(g, need, scratch, scratch_bytes, fn)) != AG_OK) return rc;
@@ -1395,7 +1280,7 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
         if ((rc = check_device_ptr(X, g->device, "X")) != AG_OK) return rc;
         if ((rc = check_device_ptr(dY, g->device, "dY")) != AG_OK) return rc;
         if ((rc = check_device_ptr(dX, g->device, "dX")) != AG_OK) return rc;
-        if (g->E > 0 && (rc = check_device_ptr(w, g->device, "w")) != AG_OK) return rc;
+        if (g->E > 0 && w && (rc = check_device_ptr(w, g->device, "w")) != AG_OK) return rc;
         if (g->E > 0 && (rc = check_device_ptr(dw, g->device, "dw")) != AG_OK) return rc;
         if (need > 0 && (rc = check_device_ptr(scratch, g->device, "scratch")) != AG_OK) return rc;
     }
@@ -1406,13 +1291,15 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
                       int64_t(s.G) * s.nv * s.vec == H;
     if (!ring || g->E == 0) {
         // shapes without the single walk: the two separate passes
-        if ((rc = spmm(g, 1, w, dY, dX, H, dtype, scratch, scratch_bytes, stream, fn, false)) != AG_OK) return rc;
-        return sddmm(g, X, dY, dw, H, dtype, scratch, scratch_bytes, stream, fn, false);
+        if ((rc = spmm(g, 1, w, dY, dX, H, dtype, scratch, scratch_bytes, stream, fn, false, mean)) != AG_OK)
+            return rc;
+        return sddmm(g, X, dY, dw, H, dtype, scratch, scratch_bytes, stream, fn, false, mean);
     }
     char *scr = static_cast<char *>(scratch);
     float *w_b = reinterpret_cast<float *>(scr + SL.w_b);
     float *dw_b = reinterpret_cast<float *>(scr + SL.dw_b);
-    regroup(true, D, w, g->E, w_b, st);
+    const EdgeScale sc = mean_scale(g, mean);
+    regroup(true, D, w, g->E, w_b, st, sc);
     Params P = base_params(g, D, H, s);
     P.order = D.bucket_of_pos;
     P.w = w_b;
@@ -1424,7 +1311,82 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
     P.n_zero = g->N - D.n_nz;
     dispatch_main<kBoth>(P, s, dtype, st);
     if (D.n_span > 0) dispatch_fixup(D, P.partial, dX, H, s, dtype, st);
-    regroup(false, D, dw_b, g->E, dw, st);
+    regroup(false, D, dw_b, g->E, dw, st, sc);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    return AG_OK;
+}
+
+// ---------------------------------------------------------------- GCN weights
+
+__global__ void k_fill(float *__restrict__ p, int64_t n, float v) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+        p[i] = v;
+}
+// unit weights: the degree is the row length of the forward CSR
+__global__ void k_row_counts(const int32_t *__restrict__ rowptr, int64_t N, float *__restrict__ deg) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < N; i += int64_t(gridDim.x) * blockDim.x)
+        deg[i] = float(rowptr[i + 1] - rowptr[i]);
+}
+// deg^-1/2 in place (0 where deg <= 0)
+__global__ void k_inv_sqrt(float *__restrict__ deg, int64_t N) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < N; i += int64_t(gridDim.x) * blockDim.x) {
+        const float d = deg[i];
+        deg[i] = d > 0.f ? 1.f / sqrtf(d) : 0.f;
+    }
+}
+// out[e] = dis[src_e] * w_e * dis[dst_e] in COO order (w = null: 1)
+__global__ void k_gcn_weights(const int32_t *__restrict__ src, const int32_t *__restrict__ dst,
+                              const float *__restrict__ w, const float *__restrict__ dis, int64_t E,
+                              float *__restrict__ out) {
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
+        const float we = w ? __ldcs(w + e) : 1.f;
+        __stcs(out + e, dis[__ldcs(src + e)] * we * dis[__ldcs(dst + e)]);
+    }
+}
+unsigned flat_grid(int64_t n) {
+    const int64_t b = (n + kThreads - 1) / kThreads;
+    return unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
+}
+
+// Scratch of ag_gcn_norm: deg[N] | ones[N] | scratch of a width-1 SpMM.
+struct GcnLayout {
+    size_t deg, ones, spmm, total;
+};
+GcnLayout gcn_layout(const ag_graph *g) {
+    GcnLayout L;
+    L.deg = 0;
+    L.ones = align_up(size_t(g->N) * 4);
+    L.spmm = L.ones + align_up(size_t(g->N) * 4);
+    L.total = L.spmm + scratch_needed(g, 1);
+    return L;
+}
+
+int gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch, size_t scratch_bytes, void *stream) {
+    const char *fn = "ag_gcn_norm";
+    if (!g) return fail(AG_ERR_INVALID_ARG, "%s: null graph", fn);
+    if (g->E > 0 && !w_norm) return fail(AG_ERR_INVALID_ARG, "%s: null w_norm", fn);
+    const GcnLayout L = gcn_layout(g);
+    int rc = check_scratch(g, L.total, scratch, scratch_bytes, fn);
+    if (rc != AG_OK) return rc;
+    if (g->E == 0) return AG_OK;
+    if ((rc = check_device_ptr(w_norm, g->device, "w_norm")) != AG_OK) return rc;
+    if (w && (rc = check_device_ptr(w, g->device, "w")) != AG_OK) return rc;
+    if ((rc = check_device_ptr(scratch, g->device, "scratch")) != AG_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *scr = static_cast<char *>(scratch);
+    float *deg = reinterpret_cast<float *>(scr + L.deg);
+    if (w) {
+        // weighted in-degree = A_w 1: the forward SpMM of a column of ones
+        float *ones = reinterpret_cast<float *>(scr + L.ones);
+        k_fill<<<flat_grid(g->N), kThreads, 0, st>>>(ones, g->N, 1.f);
+        rc = spmm(g, 0, w, ones, deg, 1, AG_F32, scr + L.spmm, scratch_bytes - L.spmm, stream, fn, false);
+        if (rc != AG_OK) return rc;
+    } else {
+        k_row_counts<<<flat_grid(g->N), kThreads, 0, st>>>(g->dir[0].rowptr, g->N, deg);
+    }
+    k_inv_sqrt<<<flat_grid(g->N), kThreads, 0, st>>>(deg, g->N);
+    k_gcn_weights<<<flat_grid(g->E), kThreads, 0, st>>>(g->coo_src, g->coo_dst, w, deg, g->E, w_norm);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
@@ -1464,6 +1426,29 @@ int ag_backward(const ag_graph *g, const float *w, const void *X, const void *dY
                 int dtype, void *scratch, size_t scratch_bytes, void *stream) {
     clear_error();
     return backward(g, w, X, dY, dX, dw, H, dtype, scratch, scratch_bytes, stream, "ag_backward", true);
+}
+
+int ag_mean_fwd(const ag_graph *g, const float *w, const void *X, void *Y, int64_t H, int dtype, void *scratch,
+                size_t scratch_bytes, void *stream) {
+    clear_error();
+    return spmm(g, 0, w, X, Y, H, dtype, scratch, scratch_bytes, stream, "ag_mean_fwd", true, true);
+}
+
+int ag_mean_backward(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw,
+                     int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream) {
+    clear_error();
+    return backward(g, w, X, dY, dX, dw, H, dtype, scratch, scratch_bytes, stream, "ag_mean_backward", true, true);
+}
+
+size_t ag_gcn_norm_scratch_bytes(const ag_graph *g) {
+    if (!g) return 0;
+    return gcn_layout(g).total;
+}
+
+int ag_gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch, size_t scratch_bytes,
+                void *stream) {
+    clear_error();
+    return gcn_norm(g, w, w_norm, scratch, scratch_bytes, stream);
 }
 
 // Staging layout: w | X | dY | Y | dX | dw | scratch, each 256-byte aligned.

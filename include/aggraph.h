@@ -208,6 +208,58 @@ AG_API int ag_backward(const ag_graph *g, const float *w, const void *X, const v
                        int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream);
 
 /*
+ * Mean aggregation (PyTorch Geometric reading guide, Step 3: the sum and mean
+ * reductions of spmm; "Done when": sum and mean are the reductions that keep
+ * the semiring structure):
+ *   Y[r] = (1 / cnt(r)) * sum over edges e into r of w_e X[src_e],
+ * cnt(r) = number of edges into r (duplicates counted), Y[r] = 0 when
+ * cnt(r) = 0.  Each edge's weight is divided by cnt(dst_e) in fp32 (IEEE
+ * division) before the same walk as ag_spmm_fwd.
+ *
+ *   w        device float [E], COO order, or NULL for unit weights
+ *   other arguments and errors as ag_spmm_fwd (same scratch size)
+ */
+AG_API int ag_mean_fwd(const ag_graph *g, const float *w, const void *X, void *Y, int64_t H, int dtype,
+                       void *scratch, size_t scratch_bytes, void *stream);
+
+/*
+ * Gradients of ag_mean_fwd for the upstream gradient dY, in one transpose
+ * walk like ag_backward:
+ *   dX[s] = sum over edges e out of s of (w_e / cnt(dst_e)) dY[dst_e]
+ *   dw_e  = dot(X[src_e], dY[dst_e]) / cnt(dst_e)
+ *
+ *   w        device float [E] (COO order) or NULL for unit weights
+ *   dw       device float [E] (COO order), or NULL: no weight gradient
+ *            (then X is not read and may be any non-NULL device pointer)
+ *   other arguments and errors as ag_backward
+ */
+AG_API int ag_mean_backward(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX,
+                            float *dw, int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
+ * GCN-normalised edge weights, D^-1/2 A_w D^-1/2 (PyTorch Geometric reading
+ * guide, "Done when": GCNConv.forward runs gcn_norm to build the normalised
+ * adjacency, then one SpMM):
+ *   deg(i)    = sum of w_e over the edges into i (w = NULL: their number)
+ *   w_norm[e] = deg(src_e)^-1/2 * w_e * deg(dst_e)^-1/2, COO order,
+ * with deg^-1/2 = 0 where deg <= 0.  Self-loops are whatever the edge list
+ * holds (add them to the COO before lowering for the usual GCN operator).
+ * The weighted degree is the forward SpMM of a column of ones (deterministic
+ * order); deg^-1/2 is 1 / sqrtf(deg), both IEEE-rounded.  Feed w_norm to
+ * ag_spmm_fwd / ag_backward.
+ *
+ *   w        device float [E] (COO order) or NULL
+ *   w_norm   device float [E], written (may be NULL when E == 0)
+ *   scratch  device buffer, 256-byte aligned, of ag_gcn_norm_scratch_bytes(g)
+ *            bytes (degrees, a column of ones and a width-1 SpMM's scratch)
+ * Errors: AG_ERR_INVALID_ARG (null graph or w_norm), AG_ERR_WORKSPACE
+ * (scratch too small or misaligned), AG_ERR_DEVICE, AG_ERR_CUDA.
+ */
+AG_API size_t ag_gcn_norm_scratch_bytes(const ag_graph *g);
+AG_API int ag_gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch, size_t scratch_bytes,
+                       void *stream);
+
+/*
  * One whole aggregation step from HOST buffers: copies w, X and dY to the
  * device staging area, runs the forward pass and the fused backward pass
  * (ag_backward), and copies Y, dX and dw back, all enqueued on `stream`.
