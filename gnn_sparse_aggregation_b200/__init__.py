@@ -25,7 +25,7 @@ import re
 import torch
 
 __all__ = ["AggraphError", "Graph", "ag_graph_lower", "ag_spmm_fwd", "ag_spmm_dx", "ag_sddmm_dw", "ag_backward",
-           "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_step_host", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
+           "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward", "ag_step_host", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
            "declared_symbols", "AG_F32", "AG_BF16"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaggraph.so")
@@ -83,6 +83,11 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_gcn_norm_scratch_bytes.argtypes = [_P]
     handle.ag_gcn_norm_scratch_bytes.restype = _SZ
     handle.ag_gcn_norm.argtypes = [_P, _P, _P, _P, _SZ, _P]
+    handle.ag_attn_scratch_bytes.argtypes = [_P, _I64]
+    handle.ag_attn_scratch_bytes.restype = _SZ
+    handle.ag_attn_fwd.argtypes = [_P, _P, _P, _P, ctypes.c_float, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_attn_backward.argtypes = [_P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P, _I64, _I, _P,
+                                        _SZ, _P]
     handle.ag_spmm_fwd_static_scratch.argtypes = [_P, _P, _P, _P, _I64, _I, _P]
     handle.ag_spmm_static_scratch_capacity.argtypes = []
     handle.ag_spmm_static_scratch_capacity.restype = _SZ
@@ -96,7 +101,7 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_status_string.restype = ctypes.c_char_p
     for name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
                  "ag_sddmm_dw", "ag_backward", "ag_spmm_fwd_static_scratch", "ag_step_host", "ag_abi_version",
-                 "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm"):
+                 "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward"):
         getattr(handle, name).restype = _I
     return handle
 
@@ -171,7 +176,7 @@ class Graph:
         st = Stats()
         _check(lib.ag_graph_get_stats(self._h, ctypes.byref(st)))
         self.stats = st.as_dict()
-        self._scratch: dict[int, torch.Tensor] = {}
+        self._scratch: dict = {}
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -361,6 +366,62 @@ def ag_gcn_norm(g: Graph, w=None, out=None, stream=None) -> torch.Tensor:
     scr = torch.empty(max(n, 1), dtype=torch.uint8, device=g.device)
     _check(lib.ag_gcn_norm(g.handle, _ptr(w), _ptr(out), _ptr(scr), n, _stream(g.device, stream)))
     return out
+
+
+def _attn_scratch(g: Graph, H: int) -> torch.Tensor:
+    n = int(lib.ag_attn_scratch_bytes(g.handle, H))
+    key = ("attn", H)
+    t = g._scratch.get(key)
+    if t is None or t.numel() < n:
+        t = torch.empty(max(n, 1), dtype=torch.uint8, device=g.device)
+        g._scratch[key] = t
+    return t
+
+
+def _same_feats(g: Graph, names, ts) -> int:
+    code = _check_feat(g, names[0], ts[0])
+    for name, t in zip(names[1:], ts[1:]):
+        if _check_feat(g, name, t) != code or t.shape != ts[0].shape:
+            raise AggraphError(2, f"{name} must match {names[0]} in shape and dtype")
+    return code
+
+
+def ag_attn_fwd(g: Graph, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: float, Y=None, alpha=None,
+                stream=None):
+    """Edge-softmax attention: (Y, alpha) with alpha in COO order."""
+    code = _same_feats(g, ("Q", "K", "V"), (Q, K, V))
+    if Y is None:
+        Y = torch.empty_like(V)
+    else:
+        _same_feats(g, ("V", "Y"), (V, Y))
+    if alpha is None:
+        alpha = torch.empty(g.E, dtype=torch.float32, device=g.device)
+    else:
+        _check_edge_vec(g, "alpha", alpha)
+    H = Q.shape[1]
+    scr = _attn_scratch(g, H)
+    _check(lib.ag_attn_fwd(g.handle, _ptr(Q), _ptr(K), _ptr(V), float(scale), _ptr(Y), _ptr(alpha), H, code,
+                           _ptr(scr), scr.numel(), _stream(g.device, stream)))
+    return Y, alpha
+
+
+def ag_attn_backward(g: Graph, Q, K, V, scale: float, alpha, dY, dQ=None, dK=None, dV=None, stream=None):
+    """Gradients (dQ, dK, dV) of ag_attn_fwd for the upstream gradient dY."""
+    code = _same_feats(g, ("Q", "K", "V", "dY"), (Q, K, V, dY))
+    _check_edge_vec(g, "alpha", alpha)
+    outs = []
+    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        if t is None:
+            t = torch.empty_like(Q)
+        else:
+            _same_feats(g, ("Q", name), (Q, t))
+        outs.append(t)
+    H = Q.shape[1]
+    scr = _attn_scratch(g, H)
+    _check(lib.ag_attn_backward(g.handle, _ptr(Q), _ptr(K), _ptr(V), float(scale), _ptr(alpha), _ptr(dY),
+                                _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), H, code, _ptr(scr), scr.numel(),
+                                _stream(g.device, stream)))
+    return tuple(outs)
 
 
 def ag_spmm_fwd_static_scratch(g: Graph, w: torch.Tensor, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:

@@ -1,0 +1,296 @@
+// Edge-softmax attention over the forward adjacency (PyTorch Geometric
+// reading guide, Step 4 "SDDMM: the second primitive, forced by attention":
+// a per-edge score from both endpoints' features, a softmax over each
+// destination row, then the SpMM with the normalised scores).
+//
+//   s_e     = scale * dot(Q[dst_e], K[src_e])           (SDDMM)
+//   alpha_e = exp(s_e - m_r) / l_r,  r = dst_e           (row softmax)
+//   Y[r]    = sum over edges e into r of alpha_e V[src_e] (SpMM)
+//
+// The scores and the two SpMMs run through this library's own entry points
+// (ag_sddmm_dw, ag_spmm_fwd, ag_spmm_dx); the row statistics m_r (maximum)
+// and l_r (sum of exp(s - m_r)) come from one segmented reduction over the
+// forward CSR, walked in the same edge-balanced tiles as the SpMM: one warp
+// per tile, a Hillis-Steele segmented scan per 32 positions, rows cut by a
+// tile boundary finished by a fixup pass in tile order.  Every reduction tree
+// is fixed by the positions alone, so results are deterministic.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "aggraph.h"
+#include "internal.h"
+
+namespace ag {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+constexpr unsigned kFull = 0xffffffffu;
+
+enum ReduceOp { kSoftmaxStats = 0, kSum = 1 };
+
+// (m, l) pairs: l is a sum of exp(value - m).  (-inf, 0) is the identity.
+__device__ __forceinline__ float2 combine_stats(float2 a, float2 b) {
+    if (a.x == -INFINITY) return b;
+    if (b.x == -INFINITY) return a;
+    const float M = fmaxf(a.x, b.x);
+    return make_float2(M, a.y * expf(a.x - M) + b.y * expf(b.x - M));
+}
+
+template <int OP>
+__device__ __forceinline__ float2 combine(float2 a, float2 b) {
+    if (OP == kSoftmaxStats) return combine_stats(a, b);
+    return make_float2(a.x + b.x, 0.f);
+}
+template <int OP>
+__device__ __forceinline__ float2 identity() {
+    return OP == kSoftmaxStats ? make_float2(-INFINITY, 0.f) : make_float2(0.f, 0.f);
+}
+
+struct ReduceParams {
+    const int32_t *order;      // forward CSR position -> COO ordinal
+    const float *a;            // COO-order inputs
+    const float *b;
+    float scale;
+    int T;                     // positions per tile
+    int64_t E, n_tiles, n_nz;
+    const int32_t *tile_nz, *nz_rows, *nz_rowptr;
+    float2 *partial;           // [2 * n_tiles]: slot 2t (row continued from the previous tile), 2t + 1 (continues)
+    float2 *out;               // [N] per row
+};
+
+__device__ __forceinline__ float2 shfl2(float2 v, int src) {
+    return make_float2(__shfl_sync(kFull, v.x, src), __shfl_sync(kFull, v.y, src));
+}
+
+// kSoftmaxStats: leaf (scale * a_e, 1); kSum: leaf (a_e * b_e, 0)
+template <int OP>
+__device__ __forceinline__ float2 leaf(const ReduceParams &P, int64_t p) {
+    const int e = __ldcs(P.order + p);
+    if (OP == kSoftmaxStats) return make_float2(P.scale * P.a[e], 1.f);
+    return make_float2(P.a[e] * P.b[e], 0.f);
+}
+
+// One warp per tile of T consecutive forward-CSR positions.  The open row
+// (nz index `cur`) holds the running aggregate `acc`; within each chunk of 32
+// positions the row starts form a lane mask and a segmented inclusive scan
+// gives every segment's aggregate at its last lane.
+template <int OP>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const ReduceParams P) {
+    const int64_t t = (int64_t(blockIdx.x) * kWarpsPerBlock) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= P.n_tiles) return;  // whole warps
+    const int64_t p0 = t * P.T;
+    const int len = int(P.E - p0 < P.T ? P.E - p0 : P.T);
+    int64_t cur = P.tile_nz[t];
+    bool before = P.nz_rowptr[cur] < p0;
+    float2 acc = identity<OP>();
+    for (int base = 0; base < len; base += 32) {
+        const int64_t cb = p0 + base;
+        const int n = len - base < 32 ? len - base : 32;
+        float2 v = lane < n ? leaf<OP>(P, cb + lane) : identity<OP>();
+        // starts of the rows after the open one that fall inside the chunk
+        unsigned bit = 0;
+        const int64_t k = cur + 1 + lane;
+        if (k < P.n_nz) {
+            const int64_t st = P.nz_rowptr[k];
+            if (st >= cb && st < cb + n) bit = 1u << int(st - cb);
+        }
+        const unsigned mask = __reduce_or_sync(kFull, bit);
+        const unsigned upto = mask & (kFull >> (31 - lane));  // heads at lanes <= this one
+        const int hs = upto ? 31 - __clz(upto) : -1;          // this lane's segment head
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            float2 o;
+            o.x = __shfl_up_sync(kFull, v.x, off);
+            o.y = __shfl_up_sync(kFull, v.y, off);
+            if (lane >= off && lane - off >= hs) v = combine<OP>(o, v);
+        }
+        const int nh = __popc(mask);
+        if (nh > 0) {
+            // the open row ends before the first head
+            const int h0 = __ffs(mask) - 1;
+            const float2 tail = shfl2(v, h0 > 0 ? h0 - 1 : 0);
+            const float2 total = h0 > 0 ? combine<OP>(acc, tail) : acc;
+            if (lane == 0) {
+                if (before) P.partial[2 * t] = total;
+                else P.out[P.nz_rows[cur]] = total;
+            }
+            // rows that start and end inside the chunk
+            const bool seg_end = lane < n - 1 && ((mask >> (lane + 1)) & 1u);
+            if (hs >= 0 && seg_end) P.out[P.nz_rows[cur + __popc(upto)]] = v;
+            // the last segment stays open
+            acc = shfl2(v, n - 1);
+            cur += nh;
+            before = false;
+        } else {
+            acc = combine<OP>(acc, shfl2(v, n - 1));
+        }
+    }
+    if (lane == 0) {
+        if (before) P.partial[2 * t] = acc;
+        else if (P.nz_rowptr[cur + 1] > p0 + len) P.partial[2 * t + 1] = acc;
+        else P.out[P.nz_rows[cur]] = acc;
+    }
+}
+
+// Rows cut by tile boundaries: out[row] = slot(2 first + 1) combined with
+// slot(2 t) for t = first + 1 .. last, in tile order (one thread per row).
+template <int OP>
+__global__ void k_row_reduce_fixup(const int4 *__restrict__ spans, int64_t n_span, const float2 *__restrict__ partial,
+                                   float2 *__restrict__ out) {
+    const int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (s >= n_span) return;
+    const int4 sp = spans[s];
+    float2 v = partial[2 * int64_t(sp.y) + 1];
+    for (int64_t t = int64_t(sp.y) + 1; t <= sp.z; ++t) v = combine<OP>(v, partial[2 * t]);
+    out[sp.x] = v;
+}
+
+// alpha_e = exp(scale * s_e - m_r) / l_r (in place over s)
+__global__ void k_softmax_alpha(float *__restrict__ s, const int32_t *__restrict__ dst, const float2 *__restrict__ ml,
+                                float scale, int64_t E) {
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
+        const float2 r = ml[__ldcs(dst + e)];
+        s[e] = expf(scale * s[e] - r.x) / r.y;
+    }
+}
+
+// ds_e = scale * alpha_e * (dalpha_e - c_r) (in place over dalpha)
+__global__ void k_attn_ds(const float *__restrict__ alpha, float *__restrict__ da, const int32_t *__restrict__ dst,
+                          const float2 *__restrict__ c, float scale, int64_t E) {
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x)
+        da[e] = scale * alpha[e] * (da[e] - c[__ldcs(dst + e)].x);
+}
+
+unsigned flat_blocks(int64_t n) {
+    const int64_t b = (n + 255) / 256;
+    return unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
+}
+
+// scratch: SpMM scratch | per-row float2 [N] | tile partials float2 [2 tiles] | float [E]
+struct AttnLayout {
+    size_t spmm, rows, partial, edges, total;
+};
+AttnLayout attn_layout(const ag_graph *g, int64_t H) {
+    AttnLayout L;
+    L.spmm = 0;
+    L.rows = align_up(ag_spmm_scratch_bytes(g, H));
+    L.partial = L.rows + align_up(size_t(g->N) * sizeof(float2));
+    L.edges = L.partial + align_up(size_t(2) * size_t(g->n_tiles) * sizeof(float2));
+    L.total = L.edges + align_up(size_t(g->E) * 4);
+    return L;
+}
+
+template <int OP>
+int row_reduce(const ag_graph *g, const float *a, const float *b, float scale, float2 *partial, float2 *out,
+               cudaStream_t st) {
+    const Direction &D = g->dir[0];
+    ReduceParams P;
+    P.order = D.order;
+    P.a = a;
+    P.b = b;
+    P.scale = scale;
+    P.T = g->tile_edges;
+    P.E = g->E;
+    P.n_tiles = g->n_tiles;
+    P.n_nz = D.n_nz;
+    P.tile_nz = D.tile_nz;
+    P.nz_rows = D.nz_rows;
+    P.nz_rowptr = D.nz_rowptr;
+    P.partial = partial;
+    P.out = out;
+    if (g->n_tiles > 0) {
+        const unsigned grid = unsigned((g->n_tiles + kWarpsPerBlock - 1) / kWarpsPerBlock);
+        k_row_reduce<OP><<<grid, kWarpsPerBlock * 32, 0, st>>>(P);
+    }
+    if (D.n_span > 0)
+        k_row_reduce_fixup<OP><<<unsigned((D.n_span + 255) / 256), 256, 0, st>>>(D.spans, D.n_span, partial, out);
+    cudaError_t err = cudaGetLastError();
+    return err == cudaSuccess ? AG_OK : cuda_fail(err, "row reduction");
+}
+
+int check_common(const ag_graph *g, int64_t H, int dtype, const void *scratch, size_t scratch_bytes, const char *fn,
+                 AttnLayout *L) {
+    if (!g) return fail(AG_ERR_INVALID_ARG, "%s: null graph", fn);
+    if (H < 1 || H > (int64_t(1) << 24)) return fail(AG_ERR_SHAPE, "%s: H = %lld outside [1, 2^24]", fn, (long long)H);
+    if (dtype != AG_F32 && dtype != AG_BF16) return fail(AG_ERR_DTYPE, "%s: unknown dtype %d", fn, dtype);
+    *L = attn_layout(g, H);
+    if (!scratch || scratch_bytes < L->total)
+        return fail(AG_ERR_WORKSPACE, "%s: scratch of %zu bytes, need %zu", fn, scratch_bytes, L->total);
+    if (reinterpret_cast<uintptr_t>(scratch) % kAlign != 0)
+        return fail(AG_ERR_WORKSPACE, "%s: scratch must be 256-byte aligned", fn);
+    return check_device_ptr(scratch, g->device, "scratch");
+}
+
+}  // namespace
+}  // namespace ag
+
+using namespace ag;
+
+extern "C" {
+
+size_t ag_attn_scratch_bytes(const ag_graph *g, int64_t H) {
+    if (!g || H < 1) return 0;
+    return attn_layout(g, H).total;
+}
+
+int ag_attn_fwd(const ag_graph *g, const void *Q, const void *K, const void *V, float scale, void *Y, float *alpha,
+                int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream) {
+    const char *fn = "ag_attn_fwd";
+    clear_error();
+    AttnLayout L;
+    int rc = check_common(g, H, dtype, scratch, scratch_bytes, fn, &L);
+    if (rc != AG_OK) return rc;
+    if (!Q || !K || !V || !Y || (g->E > 0 && !alpha)) return fail(AG_ERR_INVALID_ARG, "%s: null Q, K, V, Y or alpha", fn);
+    if (!isfinite(scale)) return fail(AG_ERR_INVALID_ARG, "%s: scale must be finite", fn);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *scr = static_cast<char *>(scratch);
+    const size_t spmm_bytes = L.rows - L.spmm;
+    if (g->E > 0) {
+        // raw scores dot(K[src], Q[dst]) in COO order, into alpha
+        if ((rc = ag_sddmm_dw(g, K, Q, alpha, H, dtype, scr + L.spmm, spmm_bytes, stream)) != AG_OK) return rc;
+        float2 *ml = reinterpret_cast<float2 *>(scr + L.rows);
+        rc = row_reduce<kSoftmaxStats>(g, alpha, nullptr, scale, reinterpret_cast<float2 *>(scr + L.partial), ml, st);
+        if (rc != AG_OK) return rc;
+        k_softmax_alpha<<<flat_blocks(g->E), 256, 0, st>>>(alpha, g->coo_dst, ml, scale, g->E);
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return cuda_fail(err, fn);
+    }
+    return ag_spmm_fwd(g, alpha, V, Y, H, dtype, scr + L.spmm, spmm_bytes, stream);
+}
+
+int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, const void *V, float scale, const float *alpha,
+                     const void *dY, void *dQ, void *dK, void *dV, int64_t H, int dtype, void *scratch,
+                     size_t scratch_bytes, void *stream) {
+    const char *fn = "ag_attn_backward";
+    clear_error();
+    AttnLayout L;
+    int rc = check_common(g, H, dtype, scratch, scratch_bytes, fn, &L);
+    if (rc != AG_OK) return rc;
+    if (!Q || !K || !V || !dY || !dQ || !dK || !dV || (g->E > 0 && !alpha))
+        return fail(AG_ERR_INVALID_ARG, "%s: null argument", fn);
+    if (!isfinite(scale)) return fail(AG_ERR_INVALID_ARG, "%s: scale must be finite", fn);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *scr = static_cast<char *>(scratch);
+    const size_t spmm_bytes = L.rows - L.spmm;
+    void *sp = scr + L.spmm;
+    // dV = A_alpha^T dY
+    if ((rc = ag_spmm_dx(g, alpha, dY, dV, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+    float *ds = reinterpret_cast<float *>(scr + L.edges);
+    if (g->E > 0) {
+        // dalpha_e = dot(V[src], dY[dst]); c_r = sum over r's edges of alpha dalpha
+        if ((rc = ag_sddmm_dw(g, V, dY, ds, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+        float2 *c = reinterpret_cast<float2 *>(scr + L.rows);
+        rc = row_reduce<kSum>(g, alpha, ds, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
+        if (rc != AG_OK) return rc;
+        k_attn_ds<<<flat_blocks(g->E), 256, 0, st>>>(alpha, ds, g->coo_dst, c, scale, g->E);
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return cuda_fail(err, fn);
+    }
+    // dQ = A_ds K (scale folded into ds), dK = A_ds^T Q
+    if ((rc = ag_spmm_fwd(g, g->E > 0 ? ds : nullptr, K, dQ, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+    return ag_spmm_dx(g, g->E > 0 ? ds : nullptr, Q, dK, H, dtype, sp, spmm_bytes, stream);
+}
+
+}  // extern "C"

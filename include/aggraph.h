@@ -260,6 +260,47 @@ AG_API int ag_gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *s
                        void *stream);
 
 /*
+ * Edge-softmax attention over the forward adjacency (PyTorch Geometric
+ * reading guide, Step 4: a per-edge score from both endpoints' features,
+ * a softmax over each destination row, then the SpMM with the normalised
+ * scores -- SpMM and SDDMM together):
+ *   s_e     = scale * dot(Q[dst_e], K[src_e])
+ *   alpha_e = exp(s_e - m_r) / sum over edges e' into r of exp(s_e' - m_r),
+ *             r = dst_e, m_r = max of s over r's edges
+ *   Y[r]    = sum over edges e into r of alpha_e V[src_e]   (0 for rows without edges)
+ * Scores are the fp32 dot products of ag_sddmm_dw; the row maximum and the
+ * sum of exponentials are reduced in fp32 in a fixed order per row; alpha
+ * is expf(s - m) / l; Y is ag_spmm_fwd with weights alpha.
+ *
+ *   Q, K, V  device [N, H] of dtype (Q gathered by destination, K and V by source)
+ *   scale    finite fp32 factor of the scores (1/sqrt(H) for scaled dot-product attention)
+ *   Y        device [N, H] of dtype, fully written
+ *   alpha    device float [E], written in COO order (kept for the backward pass)
+ *   scratch  device buffer, 256-byte aligned, of ag_attn_scratch_bytes(g, H) bytes
+ * Errors as ag_spmm_fwd; AG_ERR_INVALID_ARG also for a non-finite scale.
+ */
+AG_API size_t ag_attn_scratch_bytes(const ag_graph *g, int64_t H);
+AG_API int ag_attn_fwd(const ag_graph *g, const void *Q, const void *K, const void *V, float scale, void *Y,
+                       float *alpha, int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
+ * Gradients of ag_attn_fwd for the upstream gradient dY, by the chain rule
+ * through the row softmax:
+ *   dalpha_e = dot(dY[dst_e], V[src_e]),  c_r = sum over edges e into r of alpha_e dalpha_e
+ *   ds_e     = scale * alpha_e * (dalpha_e - c_{dst_e})
+ *   dQ[r]    = sum over edges e into r of ds_e K[src_e]        (ag_spmm_fwd with weights ds)
+ *   dK[s]    = sum over edges e out of s of ds_e Q[dst_e]      (ag_spmm_dx with weights ds)
+ *   dV[s]    = sum over edges e out of s of alpha_e dY[dst_e]  (ag_spmm_dx with weights alpha)
+ *
+ *   alpha    the alpha written by ag_attn_fwd for the same Q, K, scale
+ *   dQ, dK, dV  device [N, H] of dtype, fully written
+ *   other arguments and errors as ag_attn_fwd (same scratch size)
+ */
+AG_API int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, const void *V, float scale,
+                            const float *alpha, const void *dY, void *dQ, void *dK, void *dV, int64_t H,
+                            int dtype, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
  * One whole aggregation step from HOST buffers: copies w, X and dY to the
  * device staging area, runs the forward pass and the fused backward pass
  * (ag_backward), and copies Y, dX and dw back, all enqueued on `stream`.

@@ -72,6 +72,10 @@ def test_host_side_rejections_without_gpu(agb):
     assert lib.ag_mean_backward(None, None, None, None, None, None, 4, 0, None, 0, None) == 1
     assert lib.ag_gcn_norm(None, None, None, None, 0, None) == 1
     assert lib.ag_gcn_norm_scratch_bytes(None) == 0
+    assert lib.ag_attn_fwd(None, None, None, None, 1.0, None, None, 4, 0, None, 0, None) == 1
+    assert lib.ag_attn_backward(None, None, None, None, 1.0, None, None, None, None, None, 4, 0, None, 0,
+                                None) == 1
+    assert lib.ag_attn_scratch_bytes(None, 4) == 0
     assert lib.ag_graph_get_stats(None, None) == 1
     assert lib.ag_spmm_scratch_bytes(None, 4) == 0
     assert lib.ag_step_staging_bytes(None, 4, 0) == 0
