@@ -68,7 +68,9 @@ def _load():
                                         _P, _P, _P, _P]
         lib.oracle_attn_bwd.argtypes = [_I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_double,
                                         _P, _P, _P, _P, _P, _P]
-        for name in ("oracle_lower", "oracle_fwd", "oracle_dx", "oracle_dw",
+        lib.oracle_attn_sampled.argtypes = [_I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_double, _P,
+                                            _I64, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        for name in ("oracle_attn_sampled", "oracle_lower", "oracle_fwd", "oracle_dx", "oracle_dw",
                      "oracle_spmm_rows", "oracle_dw_edges", "oracle_mean_fwd", "oracle_mean_dx",
                      "oracle_mean_dw", "oracle_gcn_norm", "oracle_attn_fwd", "oracle_attn_bwd"):
             getattr(lib, name).restype = ctypes.c_int
@@ -257,3 +259,21 @@ def attn_bwd(src, dst, N: int, Q, K, V, scale: float, alpha, dY):
                                    float(scale), _ptr(alpha), _ptr(dY), _ptr(dQ), _ptr(dK),
                                    _ptr(dV), _ptr(ds)))
     return dQ, dK, dV, ds
+
+
+def attn_sampled(src, dst, N: int, Q, K, V, scale: float, dY, rows_r, rows_s):
+    """Y, dQ on destination rows rows_r and dK, dV on source rows rows_s of
+    the attention and its gradients, with their tolerance scales: returns a
+    dict with Y, dQ, dK, dV and absY, absdQ, absdK, absdV."""
+    src, dst = _i32(src), _i32(dst)
+    Q, K, V, dY = _f32(Q), _f32(K), _f32(V), _f32(dY)
+    rows_r, rows_s = _i32(rows_r), _i32(rows_s)
+    E = src.shape[0]
+    H = Q.shape[1]
+    r = {k: np.zeros((rows_r.shape[0], H), np.float64) for k in ("Y", "dQ", "absY", "absdQ")}
+    s = {k: np.zeros((rows_s.shape[0], H), np.float64) for k in ("dK", "dV", "absdK", "absdV")}
+    _check(_load().oracle_attn_sampled(N, E, H, _ptr(src), _ptr(dst), _ptr(Q), _ptr(K), _ptr(V), float(scale),
+                                       _ptr(dY), rows_r.shape[0], _ptr(rows_r), rows_s.shape[0], _ptr(rows_s),
+                                       _ptr(r["Y"]), _ptr(r["dQ"]), _ptr(s["dK"]), _ptr(s["dV"]),
+                                       _ptr(r["absY"]), _ptr(r["absdQ"]), _ptr(s["absdK"]), _ptr(s["absdV"])))
+    return {**r, **s}

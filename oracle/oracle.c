@@ -509,3 +509,137 @@ int oracle_attn_bwd(int64_t N, int64_t E, int64_t H, const int32_t *src, const i
     free(c);
     return ORACLE_OK;
 }
+
+/*
+ * Sampled form of the attention and its gradients for graphs too large to
+ * evaluate whole: the definitions of oracle_attn_fwd / oracle_attn_bwd,
+ * evaluated only for the destination rows sel_r (outputs Y and dQ) and the
+ * source rows sel_s (outputs dK and dV).  The row statistics m_r, l_r and
+ * c_r are formed for every row that one of those outputs needs (the sampled
+ * destinations and every destination of an edge out of a sampled source),
+ * over all of that row's edges.  Neither list may repeat a row.
+ * Scales for the tolerances: absY_r = sum over edges into r of
+ * |alpha_e V[src_e]|; with B_e = sum_h |dY[dst_e, h] V[src_e, h]| and
+ * C_r = sum over edges into r of alpha_e B_e, the weight w_e =
+ * |scale| alpha_e (B_e + C_{dst_e}) bounds |ds_e| and gives
+ * absdQ_r = sum over edges into r of w_e |K[src_e]|, absdK_s = sum over
+ * edges out of s of w_e |Q[dst_e]|, absdV_s = sum over edges out of s of
+ * alpha_e |dY[dst_e]|.
+ */
+int oracle_attn_sampled(int64_t N, int64_t E, int64_t H, const int32_t *src, const int32_t *dst,
+                        const float *Q, const float *K, const float *V, double scale, const float *dY,
+                        int64_t nsel_r, const int32_t *sel_r, int64_t nsel_s, const int32_t *sel_s,
+                        double *Y_r, double *dQ_r, double *dK_s, double *dV_s, double *absY_r,
+                        double *absdQ_r, double *absdK_s, double *absdV_s)
+{
+    if (!sizes_ok(N, E) || H < 1 || nsel_r < 0 || nsel_s < 0)
+        return ORACLE_BAD_SIZE;
+    if (!indices_ok(N, E, src, dst))
+        return ORACLE_BAD_INDEX;
+    int64_t *slot_r = (int64_t *)malloc((size_t)N * sizeof(int64_t));
+    int64_t *slot_s = (int64_t *)malloc((size_t)N * sizeof(int64_t));
+    char *need = (char *)calloc((size_t)N, 1);
+    double *m = (double *)malloc((size_t)N * sizeof(double));
+    double *z = (double *)calloc((size_t)N, sizeof(double));
+    double *c = (double *)calloc((size_t)N, sizeof(double));
+    double *C = (double *)calloc((size_t)N, sizeof(double));
+    int rc = ORACLE_OK;
+    if (!slot_r || !slot_s || !need || !m || !z || !c || !C) {
+        rc = ORACLE_NO_MEMORY;
+        goto done;
+    }
+    for (int64_t i = 0; i < N; ++i) {
+        slot_r[i] = slot_s[i] = -1;
+        m[i] = -INFINITY;
+    }
+    for (int64_t i = 0; i < nsel_r; ++i) {
+        if (sel_r[i] < 0 || sel_r[i] >= N || slot_r[sel_r[i]] >= 0) {
+            rc = ORACLE_BAD_INDEX;
+            goto done;
+        }
+        slot_r[sel_r[i]] = i;
+        need[sel_r[i]] = 1;
+    }
+    for (int64_t i = 0; i < nsel_s; ++i) {
+        if (sel_s[i] < 0 || sel_s[i] >= N || slot_s[sel_s[i]] >= 0) {
+            rc = ORACLE_BAD_INDEX;
+            goto done;
+        }
+        slot_s[sel_s[i]] = i;
+    }
+    for (int64_t e = 0; e < E; ++e)
+        if (slot_s[src[e]] >= 0)
+            need[dst[e]] = 1;
+    memset(Y_r, 0, (size_t)(nsel_r * H) * sizeof(double));
+    memset(dQ_r, 0, (size_t)(nsel_r * H) * sizeof(double));
+    memset(absY_r, 0, (size_t)(nsel_r * H) * sizeof(double));
+    memset(dK_s, 0, (size_t)(nsel_s * H) * sizeof(double));
+    memset(dV_s, 0, (size_t)(nsel_s * H) * sizeof(double));
+    memset(absdQ_r, 0, (size_t)(nsel_r * H) * sizeof(double));
+    memset(absdK_s, 0, (size_t)(nsel_s * H) * sizeof(double));
+    memset(absdV_s, 0, (size_t)(nsel_s * H) * sizeof(double));
+    /* pass 1: row maxima of the scores; pass 2: sums of exponentials */
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int64_t e = 0; e < E; ++e) {
+            const int64_t r = dst[e];
+            if (!need[r])
+                continue;
+            double acc = 0.0;
+            for (int64_t h = 0; h < H; ++h)
+                acc += (double)Q[r * H + h] * (double)K[(int64_t)src[e] * H + h];
+            const double s = scale * acc;
+            if (pass == 0) {
+                if (s > m[r])
+                    m[r] = s;
+            } else {
+                z[r] += exp(s - m[r]);
+            }
+        }
+    }
+    /* pass 3: c_r; pass 4: the outputs */
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int64_t e = 0; e < E; ++e) {
+            const int64_t r = dst[e], so = src[e];
+            if (!need[r])
+                continue;
+            double acc = 0.0, da = 0.0, B = 0.0;
+            for (int64_t h = 0; h < H; ++h) {
+                acc += (double)Q[r * H + h] * (double)K[so * H + h];
+                da += (double)dY[r * H + h] * (double)V[so * H + h];
+                B += fabs((double)dY[r * H + h] * (double)V[so * H + h]);
+            }
+            const double alpha = exp(scale * acc - m[r]) / z[r];
+            if (pass == 0) {
+                c[r] += alpha * da;
+                C[r] += alpha * B;
+                continue;
+            }
+            const double ds = alpha * (da - c[r]);
+            const double wb = fabs(scale) * alpha * (B + C[r]);
+            const int64_t i = slot_r[r], j = slot_s[so];
+            for (int64_t h = 0; h < H; ++h) {
+                if (i >= 0) {
+                    Y_r[i * H + h] += alpha * (double)V[so * H + h];
+                    absY_r[i * H + h] += fabs(alpha * (double)V[so * H + h]);
+                    dQ_r[i * H + h] += scale * ds * (double)K[so * H + h];
+                    absdQ_r[i * H + h] += wb * fabs((double)K[so * H + h]);
+                }
+                if (j >= 0) {
+                    dK_s[j * H + h] += scale * ds * (double)Q[r * H + h];
+                    dV_s[j * H + h] += alpha * (double)dY[r * H + h];
+                    absdK_s[j * H + h] += wb * fabs((double)Q[r * H + h]);
+                    absdV_s[j * H + h] += alpha * fabs((double)dY[r * H + h]);
+                }
+            }
+        }
+    }
+done:
+    free(slot_r);
+    free(slot_s);
+    free(need);
+    free(m);
+    free(z);
+    free(c);
+    free(C);
+    return rc;
+}

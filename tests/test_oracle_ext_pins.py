@@ -256,3 +256,26 @@ def test_attn_catches_planted_mistakes():
     s, _, _ = oracle.attn_fwd(src, dst, N, Q, K, K, 1.0)
     wrong = np.einsum("eh,eh->e", Q[src].astype(np.float64), K[dst])
     assert not np.allclose(s, wrong)
+
+
+def test_attn_sampled_form_matches_full():
+    rng = np.random.default_rng(17)
+    N, E, H = 30, 160, 5
+    src, dst, _, _, _ = rand_graph(rng, N, E, H)
+    Q, K, V, G = (rng.standard_normal((N, H)).astype(np.float32) for _ in range(4))
+    scale = 0.45
+    _, a, Y, bY = oracle.attn_fwd(src, dst, N, Q, K, V, scale, with_bound=True)
+    dQ, dK, dV, _ = oracle.attn_bwd(src, dst, N, Q, K, V, scale, a, G)
+    rr = np.array([0, 5, 11, int(dst[3]), 29], np.int32)
+    rr = np.unique(rr)
+    rs = np.unique(np.array([2, int(src[7]), 19, 28], np.int32))
+    o = oracle.attn_sampled(src, dst, N, Q, K, V, scale, G, rr, rs)
+    np.testing.assert_allclose(o["Y"], Y[rr], atol=1e-13)
+    np.testing.assert_allclose(o["absY"], bY[rr], atol=1e-13)
+    np.testing.assert_allclose(o["dQ"], dQ[rr], atol=1e-13)
+    np.testing.assert_allclose(o["dK"], dK[rs], atol=1e-13)
+    np.testing.assert_allclose(o["dV"], dV[rs], atol=1e-13)
+    # the gradient scales dominate the gradients they bound
+    assert (np.abs(o["dQ"]) <= o["absdQ"] + 1e-12).all()
+    assert (np.abs(o["dK"]) <= o["absdK"] + 1e-12).all()
+    assert (np.abs(o["dV"]) <= o["absdV"] + 1e-12).all()
