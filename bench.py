@@ -54,6 +54,8 @@ def parse_args():
                    help="override the R-MAT scale (smaller cases for profiling)")
     p.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-rows", action="store_true",
+                   help="skip the timings of mean, GCN weights and attention reported beside the step")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time per sample")
     return p.parse_args()
 
@@ -79,6 +81,21 @@ def algorithmic_bytes(N, E, H, elem):
     dw = 8 * E + 4 * E + 2 * N * H * elem
     backward = 4 * (N + 1) + 4 * E + 4 * E + 4 * E + 4 * E + 3 * N * H * elem
     return {"fwd": spmm, "dx": spmm, "dw": dw, "backward": backward}
+
+
+def row_bytes(N, E, H, elem):
+    """Minimal bytes of one call of the further aggregators: mean as the
+    weighted sum; GCN weights read the forward row pointers and both COO
+    index arrays and write the weights; attention forward reads the forward
+    CSR (row pointers, columns, order map), Q, K and V once and writes Y and
+    alpha; its backward reads both CSRs, alpha, Q, K, V and dY once and writes
+    dQ, dK and dV."""
+    algo = algorithmic_bytes(N, E, H, elem)
+    csr = 4 * (N + 1) + 8 * E
+    return {"mean_fwd": algo["fwd"], "mean_backward": algo["backward"],
+            "gcn_norm": 4 * (N + 1) + 8 * E + 4 * E,
+            "attn_fwd": csr + 4 * E + 4 * N * H * elem,
+            "attn_backward": 2 * csr + 4 * E + 7 * N * H * elem}
 
 
 def launches_per_step_of(st, wl):
@@ -365,6 +382,32 @@ def our_arm(args):
     per_op["dx"] = timed(lambda: agb.ag_spmm_dx(g, wl.w, wl.dY, dX), K)
     per_op["dw"] = timed(lambda: agb.ag_sddmm_dw(g, wl.X, wl.dY, dw), K)
 
+    # the further aggregators on the same graph (reported beside the step, not in it)
+    rows = {}
+    if not args.no_rows:
+        Kr = max(3, min(K, 10))
+        mk = lambda s: workloads.features(wl.N, wl.H, wl.feature_dtype, 11000 + s, dev)
+        Q, Kf, V = mk(1), mk(2), mk(3)
+        Ya, dQ, dK, dV = (torch.empty_like(wl.X) for _ in range(4))
+        alpha = torch.empty(wl.E, dtype=torch.float32, device=dev)
+        scale = 1.0 / wl.H ** 0.5
+        wn = torch.empty_like(wl.w)
+        calls = {
+            "mean_fwd": lambda: agb.ag_mean_fwd(g, wl.w, wl.X, Y),
+            "mean_backward": lambda: agb.ag_mean_backward(g, wl.w, wl.X, wl.dY, dX, dw),
+            "gcn_norm": lambda: agb.ag_gcn_norm(g, None, wn),
+            "attn_fwd": lambda: agb.ag_attn_fwd(g, Q, Kf, V, scale, Ya, alpha),
+            "attn_backward": lambda: agb.ag_attn_backward(g, Q, Kf, V, scale, alpha, wl.dY, dQ, dK, dV),
+        }
+        rb = row_bytes(wl.N, wl.E, wl.H, wl.X.element_size())
+        for name, fn in calls.items():
+            t = timed(fn, Kr)
+            avg_ms = sum(t) / len(t)
+            gbs = rb[name] / (avg_ms / 1e3) / 1e9
+            rows[name] = {"ms": avg_ms, "algorithmic_bytes": rb[name], "GB_per_s": gbs,
+                          "frac_of_peak": gbs / peaks()[0], "calls": Kr}
+        del Q, Kf, V, Ya, dQ, dK, dV, alpha, wn
+
     # end to end from host buffers, copies inside the timed region
     e2e = None
     Ke = args.e2e_steps if args.e2e_steps is not None else min(K, 5)
@@ -423,6 +466,7 @@ def our_arm(args):
                                         "spanning_rows_t", "long_spanning_rows_t", "max_degree_f",
                                         "max_degree_t")},
         "gpu_launches": launches_per_step * K,
+        "rows": rows,
         "clocks": clocks,
         "e2e": e2e,
     }
