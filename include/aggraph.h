@@ -146,8 +146,8 @@ AG_API int ag_graph_get_stats(const ag_graph *g, ag_graph_stats *out);
 AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
 
 /*
- * Forward aggregation Y = A_w X ("Decision": forward reuses the
- * destination-owned CSR traversal; reading guide Step 3: the gather / message /
+ * Forward aggregation Y = A_w X ("Decision": the forward pass walks the CSR
+ * whose rows belong to destinations; reading guide Step 3: the gather / message /
  * scatter triple is one SpMM when the message is a scalar multiple of the
  * source row, PyG GraphConv's edge_weight * x_j of section "Reference
  * contract").
