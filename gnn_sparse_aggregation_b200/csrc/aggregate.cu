@@ -1451,6 +1451,55 @@ int ag_gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch,
     return gcn_norm(g, w, w_norm, scratch, scratch_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+// Two helper streams per device for ag_step_host (created once, never
+// destroyed): one brings dY in while the forward pass runs, one takes the
+// results out, so that host-to-device and device-to-host copies overlap.
+constexpr int kStepDevices = 64;
+std::mutex g_step_mu;
+cudaStream_t g_step_in[kStepDevices] = {}, g_step_out[kStepDevices] = {};
+
+int step_streams(int device, cudaStream_t *in, cudaStream_t *out) {
+    if (device < 0 || device >= kStepDevices) return fail(AG_ERR_DEVICE, "ag_step_host: device %d", device);
+    std::lock_guard<std::mutex> lock(g_step_mu);
+    if (!g_step_in[device]) {
+        cudaStream_t a = nullptr, b = nullptr;
+        cudaError_t err = cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking);
+        if (err == cudaSuccess) err = cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking);
+        if (err != cudaSuccess) {
+            if (a) cudaStreamDestroy(a);
+            return cuda_fail(err, "ag_step_host: stream creation");
+        }
+        g_step_in[device] = a;
+        g_step_out[device] = b;
+    }
+    *in = g_step_in[device];
+    *out = g_step_out[device];
+    return AG_OK;
+}
+
+// Events of one ag_step_host call, released when the call returns (the
+// runtime keeps them alive until the work that waits on them is done).
+struct StepEvents {
+    cudaEvent_t e[5] = {};
+    cudaError_t create() {
+        for (auto &x : e) {
+            cudaError_t err = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+            if (err != cudaSuccess) return err;
+        }
+        return cudaSuccess;
+    }
+    ~StepEvents() {
+        for (auto &x : e)
+            if (x) cudaEventDestroy(x);
+    }
+};
+}  // namespace
+
+extern "C" {
+
 // Staging layout: w | X | dY | Y | dX | dw | scratch, each 256-byte aligned.
 static bool staging_layout(const ag_graph *g, int64_t H, int dtype, size_t off[7], size_t *total) {
     if (!g || H < 1 || (dtype != AG_F32 && dtype != AG_BF16)) return false;
@@ -1494,22 +1543,44 @@ int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, con
     const size_t feat = size_t(g->N) * size_t(H) * (dtype == AG_F32 ? 4 : 2);
     const size_t wb = size_t(g->E) * 4;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t err = cudaSuccess;
-    auto copy = [&](void *to, const void *from, size_t n, cudaMemcpyKind k) {
-        if (err == cudaSuccess && n > 0) err = cudaMemcpyAsync(to, from, n, k, st);
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    if ((rc = step_streams(g->device, &s_in, &s_out)) != AG_OK) return rc;
+    StepEvents ev;
+    cudaError_t err = ev.create();
+    auto copy = [&](void *to, const void *from, size_t n, cudaMemcpyKind k, cudaStream_t s) {
+        if (err == cudaSuccess && n > 0) err = cudaMemcpyAsync(to, from, n, k, s);
+    };
+    auto record = [&](cudaEvent_t e, cudaStream_t s) {
+        if (err == cudaSuccess) err = cudaEventRecord(e, s);
+    };
+    auto wait = [&](cudaStream_t s, cudaEvent_t e) {
+        if (err == cudaSuccess) err = cudaStreamWaitEvent(s, e, 0);
     };
     const size_t scr = scratch_needed(g, H);  // staging's scratch part
-    copy(w, w_host, wb, cudaMemcpyHostToDevice);
-    copy(X, X_host, feat, cudaMemcpyHostToDevice);
+    // w and X first; dY follows on its own stream while the forward pass runs
+    copy(w, w_host, wb, cudaMemcpyHostToDevice, st);
+    copy(X, X_host, feat, cudaMemcpyHostToDevice, st);
+    record(ev.e[0], st);
+    wait(s_in, ev.e[0]);
+    copy(dY, dY_host, feat, cudaMemcpyHostToDevice, s_in);
+    record(ev.e[1], s_in);
     if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy in");
     if ((rc = spmm(g, 0, w, X, Y, H, dtype, scratch, scr, stream, "ag_step_host", false)) != AG_OK) return rc;
-    copy(Y_host, Y, feat, cudaMemcpyDeviceToHost);
-    copy(dY, dY_host, feat, cudaMemcpyHostToDevice);
+    // Y goes out (device to host) while dY still comes in (host to device)
+    record(ev.e[2], st);
+    wait(s_out, ev.e[2]);
+    copy(Y_host, Y, feat, cudaMemcpyDeviceToHost, s_out);
+    wait(st, ev.e[1]);
     if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy");
     if ((rc = backward(g, w, X, dY, dX, dw, H, dtype, scratch, scr, stream, "ag_step_host", false)) != AG_OK)
         return rc;
-    copy(dX_host, dX, feat, cudaMemcpyDeviceToHost);
-    copy(dw_host, dw, wb, cudaMemcpyDeviceToHost);
+    record(ev.e[3], st);
+    wait(s_out, ev.e[3]);
+    copy(dX_host, dX, feat, cudaMemcpyDeviceToHost, s_out);
+    copy(dw_host, dw, wb, cudaMemcpyDeviceToHost, s_out);
+    // `stream` covers every copy: the caller synchronizes it alone
+    record(ev.e[4], s_out);
+    wait(st, ev.e[4]);
     if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy out");
     return AG_OK;
 }

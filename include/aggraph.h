@@ -303,7 +303,11 @@ AG_API int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, con
 /*
  * One whole aggregation step from HOST buffers: copies w, X and dY to the
  * device staging area, runs the forward pass and the fused backward pass
- * (ag_backward), and copies Y, dX and dw back, all enqueued on `stream`.
+ * (ag_backward), and copies Y, dX and dw back.  The copy of dY and the copies
+ * out run on two helper streams of the graph's device (created on first use,
+ * kept until exit) and are joined to `stream` with events, so that dY comes
+ * in while the forward pass runs and Y goes out while dY comes in; `stream`
+ * is ordered after every one of them.
  *
  *   *_host   host buffers (page-locked memory is needed for the copies to be
  *            asynchronous); w_host/dw_host may be NULL when E == 0

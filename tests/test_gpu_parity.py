@@ -278,6 +278,33 @@ def test_step_from_host_buffers(agb, dtype):
     assert torch.equal(hY, Y.cpu()) and torch.equal(hdX, dX.cpu()) and torch.equal(hdw, dw.cpu())
 
 
+def test_step_from_host_buffers_orders_on_the_callers_stream(agb):
+    # three steps back to back on one side stream, sharing one staging
+    # buffer; only that stream is synchronized, so every copy (including those
+    # on the library's helper streams) must be ordered before it
+    N, src, dst = skewed_edges(N=1500, E=20000)
+    wl, g = graph(agb, N, src, dst, 32, torch.bfloat16)
+    staging = torch.empty(agb.ag_step_staging_bytes(g, wl.H, torch.bfloat16), dtype=torch.uint8, device=DEV)
+    ins, outs, refs = [], [], []
+    for k in range(3):
+        w = wl.w * (k + 1)
+        X = (wl.X.float() - k).bfloat16()
+        dY = (wl.dY.float() + k).bfloat16()
+        refs.append(tuple(t.cpu() for t in (g.fwd(w, X), *g.backward(w, X, dY))))
+        ins.append(tuple(t.cpu().pin_memory() for t in (w, X, dY)))
+        outs.append((torch.empty_like(ins[-1][1]).pin_memory(), torch.empty_like(ins[-1][1]).pin_memory(),
+                     torch.empty_like(ins[-1][0]).pin_memory()))
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    for (hw, hX, hdY), (hY, hdX, hdw) in zip(ins, outs):
+        agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging, stream=s)
+    s.synchronize()
+    for (hY, hdX, hdw), (Y, dX, dw) in zip(outs, refs):
+        assert torch.equal(hY.view(torch.int16), Y.view(torch.int16))
+        assert torch.equal(hdX.view(torch.int16), dX.view(torch.int16))
+        assert torch.equal(hdw, dw)
+
+
 def test_errors_are_reported_not_launched(agb):
     N, src, dst = skewed_edges(N=300, E=2000)
     wl, g = graph(agb, N, src, dst, 8)
