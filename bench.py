@@ -114,7 +114,7 @@ def source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gnn_sparse_aggregation_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".h")):
+        if fn.endswith((".cu", ".cuh", ".h")):
             with open(os.path.join(csrc, fn), "rb") as f:
                 h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]

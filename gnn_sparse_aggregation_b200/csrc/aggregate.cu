@@ -1,28 +1,35 @@
 // aggregate.cu -- per-call kernels: weighted SpMM (forward Y = A_w X and
-// feature gradient dX = A_w^T dY) and the per-edge SDDMM weight gradient
-// dw_e = dot(X[src_e], dY[dst_e]).
+// feature gradient dX = A_w^T dY), the per-edge SDDMM weight gradient
+// dw_e = dot(X[src_e], dY[dst_e]), both gradients in one walk, the mean
+// aggregation and the GCN-normalised weights.
 //
 // tinymesh "Weighted aggregation experiment", section "Decision": forward and
-// dX reuse one owner-row CSR traversal, dw has one output per edge reduced
-// over the feature width, and none of them needs atomics or an [E, H]
-// intermediate.  Section "Limits" names the two weak spots of that design:
-// a serial reduction over the feature width per edge, and degree skew in the
-// CSR directions.  Here:
-//   * an owner row is handled by a group of G lanes that together span the
-//     feature width with 16-byte vector loads (float4 / 8 x bf16), several
-//     gathered rows in flight per lane, fp32 accumulation in registers;
-//   * rows come in decreasing-degree order (longest work first), and rows
-//     longer than kHeavyThreshold are cut into kChunkEdges-edge chunks whose
-//     fp32 partial rows go to caller scratch and are summed in chunk order by
-//     a second kernel -- deterministic, no float atomics;
-//   * dw walks the transpose CSR: the owner's X row is held in registers and
-//     every dY row gathered once feeds one dot product, reduced across the
-//     group with xor shuffles.
+// dX use owner-row CSR traversals, dw has one output per edge reduced over the
+// feature width, and none of them needs atomics or an [E, H] intermediate.
+// Section "Limits" names the two weak spots of that design: a serial
+// reduction over the feature width per edge, and degree skew in the CSR
+// directions.  Here:
+//   * the CSR positions are cut into edge-balanced tiles of T positions; a
+//     group of G lanes walks one tile, each lane owning 16-byte vectors of
+//     the feature width, gathered rows in flight through a per-lane
+//     shared-memory ring filled with cp.async, fp32 accumulation in
+//     registers;
+//   * a row cut by tile boundaries leaves fp32 partial rows in caller scratch
+//     that a second kernel adds in tile order -- deterministic, no float
+//     atomics;
+//   * the per-call weights (COO order) are first regrouped into windows of
+//     2^20 CSR positions, so the walk reads them from L2, and the weight
+//     gradient leaves through the same windows back to COO order;
+//   * dw walks the transpose CSR: the owner's X row is held in registers,
+//     every dY row gathered once feeds one dot product, and the dots of a
+//     chunk of positions are reduced across the group with one
+//     reduce-scatter.
 #include <cuda_bf16.h>
 
 #include <climits>
 #include <mutex>
 
+#include "device_common.cuh"
 #include "internal.h"
 
 namespace ag {
@@ -31,9 +38,6 @@ namespace {
 // Tunables (compile-time; the defaults are the measured best on B200).
 #ifndef AG_RING_DEPTH
 #define AG_RING_DEPTH 8   // gathered rows in flight per lane group (shared-memory ring)
-#endif
-#ifndef AG_RING_L1
-#define AG_RING_L1 0      // 1: ring copies also allocate in L1 (cp.async.ca), 0: L2 only (.cg)
 #endif
 #ifndef AG_W_STREAM
 #define AG_W_STREAM 0     // 1: weight lookups loaded evict-first; 0: normal caching (the bucketed
@@ -59,78 +63,6 @@ constexpr int kRingDepth = AG_RING_DEPTH;
 constexpr int kChunk = AG_CHUNK;
 
 enum Mode { kSpmm = 1, kSddmm = 2, kBoth = 3 };  // kBoth: feature and weight gradient in one walk
-
-using bf16_t = uint16_t;  // bfloat16 stored as raw bits
-
-__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
-__device__ __forceinline__ uint32_t bf16_bits(float f) {
-    return uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) { return bf16_bits(a) | (bf16_bits(b) << 16); }
-
-// Vector access to VEC consecutive features: gathered rows stay in their
-// storage type ("raw") until they are used, so that several rows in flight
-// cost only their own size in registers.
-template <typename T, int VEC> struct Vec;
-
-template <> struct Vec<float, 4> {
-    using raw = float4;
-    static __device__ __forceinline__ raw zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-    static __device__ __forceinline__ raw load_raw(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
-    static __device__ __forceinline__ void unpack(raw t, float (&v)[4]) { v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w; }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
-        __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
-    }
-};
-template <> struct Vec<float, 1> {
-    using raw = float;
-    static __device__ __forceinline__ raw zero() { return 0.f; }
-    static __device__ __forceinline__ raw load_raw(const float *p) { return __ldg(p); }
-    static __device__ __forceinline__ void unpack(raw t, float (&v)[1]) { v[0] = t; }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[1]) { __stcs(p, v[0]); }
-};
-template <> struct Vec<bf16_t, 8> {
-    using raw = uint4;
-    static __device__ __forceinline__ raw zero() { return make_uint4(0u, 0u, 0u, 0u); }
-    static __device__ __forceinline__ raw load_raw(const bf16_t *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
-    static __device__ __forceinline__ void unpack(raw t, float (&v)[8]) {
-        v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
-        v[4] = bf16_lo(t.z); v[5] = bf16_hi(t.z); v[6] = bf16_lo(t.w); v[7] = bf16_hi(t.w);
-    }
-    static __device__ __forceinline__ void store(bf16_t *p, const float (&v)[8]) {
-        uint4 t = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                             pack_bf16(v[6], v[7]));
-        __stcs(reinterpret_cast<uint4 *>(p), t);
-    }
-};
-template <> struct Vec<bf16_t, 2> {
-    using raw = uint32_t;
-    static __device__ __forceinline__ raw zero() { return 0u; }
-    static __device__ __forceinline__ raw load_raw(const bf16_t *p) {
-        return __ldg(reinterpret_cast<const unsigned int *>(p));
-    }
-    static __device__ __forceinline__ void unpack(raw t, float (&v)[2]) { v[0] = bf16_lo(t); v[1] = bf16_hi(t); }
-    static __device__ __forceinline__ void store(bf16_t *p, const float (&v)[2]) {
-        __stcs(reinterpret_cast<unsigned int *>(p), pack_bf16(v[0], v[1]));
-    }
-};
-template <> struct Vec<bf16_t, 1> {
-    using raw = uint32_t;
-    static __device__ __forceinline__ raw zero() { return 0u; }
-    static __device__ __forceinline__ raw load_raw(const bf16_t *p) {
-        return uint32_t(__ldg(reinterpret_cast<const unsigned short *>(p)));
-    }
-    static __device__ __forceinline__ void unpack(raw t, float (&v)[1]) { v[0] = __uint_as_float(t << 16); }
-    static __device__ __forceinline__ void store(bf16_t *p, const float (&v)[1]) {
-        *reinterpret_cast<unsigned short *>(p) = (unsigned short)bf16_bits(v[0]);
-    }
-};
-
-template <typename T, int VEC>
-__device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
-    Vec<T, VEC>::unpack(Vec<T, VEC>::load_raw(p), v);
-}
 
 // A weight looked up through the bucketed layout: each 128-byte line of a
 // window is used by about 32 positions of that window's tiles, so it is kept
@@ -382,20 +314,6 @@ k_tiles(const Params P) {
 
 // ---------------------------------------------------------------------------- shared-memory ring path
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-#if AG_RING_L1
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-#else
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-#endif
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-
 template <typename T, int VEC>
 __device__ __forceinline__ typename Vec<T, VEC>::raw lds_raw(const uint4 *p) {
     if constexpr (sizeof(typename Vec<T, VEC>::raw) == 16) {
@@ -451,33 +369,6 @@ __device__ __forceinline__ float reduce_chunk(float (&v)[U], int gl, unsigned gm
 #pragma unroll
     for (int o = U; o < G; o <<= 1) v[0] += __shfl_xor_sync(gmask, v[0], o, G);
     return v[0];
-}
-
-// dot product of two raw 16-byte vectors, accumulated in order into c.
-// bf16: fma.rn.f32.bf16 multiplies two bf16 values exactly and adds in fp32
-// with one rounding -- the same result as widening both to fp32 first.
-__device__ __forceinline__ float dot_raw(float4 a, float4 b, float c) {
-    c = fmaf(a.x, b.x, c);
-    c = fmaf(a.y, b.y, c);
-    c = fmaf(a.z, b.z, c);
-    return fmaf(a.w, b.w, c);
-}
-__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float c) {
-    float d;
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
-        "mov.b32 {al, ah}, %1;\n\t"
-        "mov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t"
-        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
-        : "=f"(d)
-        : "r"(a), "r"(b), "f"(c));
-    return d;
-}
-__device__ __forceinline__ float dot_raw(uint4 a, uint4 b, float c) {
-    c = dot2_bf16(a.x, b.x, c);
-    c = dot2_bf16(a.y, b.y, c);
-    c = dot2_bf16(a.z, b.z, c);
-    return dot2_bf16(a.w, b.w, c);
 }
 
 // Row accumulator of one lane: NV vectors of VEC fp32 sums updated with
