@@ -109,6 +109,18 @@ def test_attention_matches_oracle(agb, name, dtype):
     assert torch.allclose(sums[has], torch.ones_like(sums[has]), atol=1e-5)
 
 
+@pytest.mark.parametrize("H,dtype", [(1, torch.float32), (3, torch.float32), (8, torch.bfloat16),
+                                     (33, torch.float32), (40, torch.bfloat16)])
+def test_attention_narrow_and_ragged_widths(agb, H, dtype):
+    # widths that take the register (non-ring) walks and ragged vector tails
+    rng = np.random.default_rng(H)
+    N, E = 700, 6000
+    src = np.concatenate([rng.integers(0, N, E), rng.integers(0, N, 900)])
+    dst = np.concatenate([rng.integers(0, N // 2, E), np.full(900, 5)])
+    wl = workloads.custom(N, src, dst, H, seed=H, device=DEV)
+    _check_attention(agb, wl, dtype, f"H={H}/{dtype}")
+
+
 def test_attention_skewed_rows_cut_by_many_tiles(agb):
     # one destination with 40,000 inputs (cut into many tiles), a few light
     # rows, empty rows and duplicate edges

@@ -81,6 +81,30 @@ def test_mean_unit_weights(agb, config):
     assert_within(dw, rw, bw, TOL_DW, f"{wl.name} unit mean dw")
 
 
+@pytest.mark.parametrize("H,dtype", [(1, torch.float32), (5, torch.bfloat16), (17, torch.float32),
+                                     (96, torch.bfloat16)])
+def test_mean_narrow_and_ragged_widths(agb, H, dtype):
+    import oracle
+    rng = np.random.default_rng(100 + H)
+    N, E = 800, 7000
+    src = np.concatenate([rng.integers(0, N, E), np.full(1200, 9)])
+    dst = np.concatenate([rng.integers(0, N, E), rng.integers(0, 40, 1200)])
+    wl = workloads.custom(N, src, dst, H, seed=H, feature_dtype=dtype, device=DEV)
+    g = agb.ag_graph_lower(wl.src, wl.dst, N)
+    Y = agb.ag_mean_fwd(g, wl.w, wl.X)
+    dX, dw = agb.ag_mean_backward(g, wl.w, wl.X, wl.dY)
+    torch.cuda.synchronize()
+    s, d = host(wl.src), host(wl.dst)
+    hw, hX, hdY = host(wl.w), host(wl.X), host(wl.dY)
+    tol = TOL[dtype]
+    rY, bY = oracle.mean_fwd(s, d, N, hw, hX, with_bound=True)
+    rX, bX = oracle.mean_dx(s, d, N, hw, hdY, with_bound=True)
+    rw, bw = oracle.mean_dw(s, d, N, hX, hdY, with_bound=True)
+    assert_within(Y, rY, bY, tol, f"H={H} mean Y")
+    assert_within(dX, rX, bX, tol, f"H={H} mean dX")
+    assert_within(dw, rw, bw, TOL_DW, f"H={H} mean dw")
+
+
 def test_mean_of_unit_in_degree_equals_weighted_sum(agb):
     # every node receives exactly one edge: mean == sum, bit for bit
     N, H = 3000, 64
