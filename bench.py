@@ -110,13 +110,17 @@ def launches_per_step_of(st, wl):
     return fwd + bwd
 
 
+STEP_SOURCES = ("aggregate.cu", "device_common.cuh", "internal.h", "lower.cu")
+
+
 def source_hash():
+    """Hash of the sources of the step's kernels and of the schedule they walk
+    (a traffic record taken on other sources is not reported)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gnn_sparse_aggregation_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + f.read())
+    for fn in STEP_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 

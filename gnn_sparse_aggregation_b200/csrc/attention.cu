@@ -7,8 +7,9 @@
 //   alpha_e = exp(s_e - m_r) / l_r,  r = dst_e           (row softmax)
 //   Y[r]    = sum over edges e into r of alpha_e V[src_e] (SpMM)
 //
-// The scores and the two SpMMs run through this library's own entry points
-// (ag_sddmm_dw, ag_spmm_fwd, ag_spmm_dx); the row statistics m_r (maximum)
+// The scores and the SpMMs run through this library's own entry points
+// (ag_sddmm_dw, ag_spmm_fwd, ag_spmm_dx, and ag_backward for dV with dalpha
+// in one walk); the row statistics m_r (maximum)
 // and l_r (sum of exp(s - m_r)) come from one segmented reduction over the
 // forward CSR, walked in the same edge-balanced tiles as the SpMM: one warp
 // per tile, a Hillis-Steele segmented scan per 32 positions, rows cut by a
@@ -275,12 +276,14 @@ int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, const void
     char *scr = static_cast<char *>(scratch);
     const size_t spmm_bytes = L.rows - L.spmm;
     void *sp = scr + L.spmm;
-    // dV = A_alpha^T dY
-    if ((rc = ag_spmm_dx(g, alpha, dY, dV, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
     float *ds = reinterpret_cast<float *>(scr + L.edges);
-    if (g->E > 0) {
-        // dalpha_e = dot(V[src], dY[dst]); c_r = sum over r's edges of alpha dalpha
-        if ((rc = ag_sddmm_dw(g, V, dY, ds, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+    if (g->E == 0) {
+        if ((rc = ag_spmm_dx(g, alpha, dY, dV, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+    } else {
+        // dV = A_alpha^T dY and dalpha_e = dot(V[src], dY[dst]) in one transpose
+        // walk (the weighted-sum backward with weights alpha and "features" V)
+        if ((rc = ag_backward(g, alpha, V, dY, dV, ds, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+        // c_r = sum over r's edges of alpha dalpha
         float2 *c = reinterpret_cast<float2 *>(scr + L.rows);
         rc = row_reduce<kSum>(g, alpha, ds, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
         if (rc != AG_OK) return rc;

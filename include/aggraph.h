@@ -290,7 +290,8 @@ AG_API int ag_attn_fwd(const ag_graph *g, const void *Q, const void *K, const vo
  *   ds_e     = scale * alpha_e * (dalpha_e - c_{dst_e})
  *   dQ[r]    = sum over edges e into r of ds_e K[src_e]        (ag_spmm_fwd with weights ds)
  *   dK[s]    = sum over edges e out of s of ds_e Q[dst_e]      (ag_spmm_dx with weights ds)
- *   dV[s]    = sum over edges e out of s of alpha_e dY[dst_e]  (ag_spmm_dx with weights alpha)
+ *   dV[s]    = sum over edges e out of s of alpha_e dY[dst_e]  (with dalpha: ag_backward with
+ *                                                               weights alpha and features V)
  *
  *   alpha    the alpha written by ag_attn_fwd for the same Q, K, scale
  *   dQ, dK, dV  device [N, H] of dtype, fully written
