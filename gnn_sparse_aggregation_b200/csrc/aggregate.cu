@@ -408,14 +408,15 @@ template <typename T, int NV, int VEC> struct RowAcc {
 // (groups [n_tiles, n_tiles_pad) are idle fillers), every group of a warp
 // runs the warp's longest tile length in batches of G positions with its own
 // bounds as predicates, and the shuffles of the common path use the full
-// warp mask.  A batch inside every group's tile runs fully unrolled without
-// bounds checks (slots, shuffle lanes and refill sources are constants).
-// Indices are prefetched two batches ahead and weights one batch ahead.
-// kSddmm reduces the G dot products of an unrolled batch with one
-// reduce-scatter, after which lane j writes the weight gradient of the
-// batch's position j.  kBoth does both on one walk of the transpose CSR: each
+// warp mask.  A batch inside every group's tile runs without bounds checks:
+// fully unrolled in the forward walk, in rolled chunks of U unrolled
+// positions in the gradient walks (slots, shuffle lanes and refill sources
+// are constants within a chunk).  Indices are prefetched two batches ahead
+// and weights one batch ahead.  kSddmm reduces the U dot products of a chunk
+// with one reduce-scatter, after which the lane of each position writes its
+// weight gradient.  kBoth does both on one walk of the transpose CSR: each
 // gathered dY row feeds the feature-gradient row of its source and the dot
-// product of its edge.  Rows are accumulated with packed fp32 pairs.
+// product of its edge.  Rows are accumulated with scalar fp32 FMAs.
 template <typename T, int VEC, int NV, int G, int MODE, int D>
 __global__ void __launch_bounds__(kThreads)
 k_tiles_ring(const Params P) {
