@@ -26,6 +26,7 @@
 //     reduce-scatter.
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <climits>
 #include <mutex>
 
@@ -798,11 +799,16 @@ void launch_ring(const Params &P, cudaStream_t st) {
     const unsigned grid = unsigned((groups + kThreads / G - 1) / (kThreads / G));
     // ring: D slots x NV vectors x 16 bytes for every lane of the block
     const size_t smem = size_t(kThreads) * D * NV * 16;
-    static bool configured = false;  // per instantiation: the attribute belongs to the function
-    if (!configured) {
+    // the shared-memory limit is an attribute of the function in each device's
+    // context: set it once per device (a race only repeats the same call)
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = uint64_t(1) << (dev & 63);
+    if (!(configured.load(std::memory_order_relaxed) & bit)) {
         cudaFuncSetAttribute(k_tiles_ring<T, VEC, NV, G, MODE, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
-        configured = true;
+        configured.fetch_or(bit, std::memory_order_relaxed);
     }
     k_tiles_ring<T, VEC, NV, G, MODE, D><<<grid, kThreads, smem, st>>>(P);
 }
@@ -904,7 +910,7 @@ int check_call(const ag_graph *g, int64_t H, int dtype, const char *fn) {
     if (dtype != AG_F32 && dtype != AG_BF16) return fail(AG_ERR_DTYPE, "%s: unknown dtype %d", fn, dtype);
     if (H < 1 || H > (int64_t(1) << 24) || g->N * H >= (int64_t(1) << 40))
         return fail(AG_ERR_SHAPE, "%s: H=%lld out of range for N=%lld", fn, (long long)H, (long long)g->N);
-    return AG_OK;
+    return check_current_device(g, fn);
 }
 
 // Per-call scratch: [partial rows][weights, bucketed][weight gradient, bucketed]
@@ -1257,6 +1263,7 @@ GcnLayout gcn_layout(const ag_graph *g) {
 int gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch, size_t scratch_bytes, void *stream) {
     const char *fn = "ag_gcn_norm";
     if (!g) return fail(AG_ERR_INVALID_ARG, "%s: null graph", fn);
+    if (int rc0 = check_current_device(g, fn)) return rc0;
     if (g->E > 0 && !w_norm) return fail(AG_ERR_INVALID_ARG, "%s: null w_norm", fn);
     const GcnLayout L = gcn_layout(g);
     int rc = check_scratch(g, L.total, scratch, scratch_bytes, fn);

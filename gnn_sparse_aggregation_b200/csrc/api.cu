@@ -25,6 +25,15 @@ int cuda_fail(cudaError_t err, const char *what) {
 
 void clear_error() { g_err[0] = '\0'; }
 
+int check_current_device(const ag_graph *g, const char *fn) {
+    int cur = -1;
+    cudaError_t err = cudaGetDevice(&cur);
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    if (cur != g->device)
+        return fail(AG_ERR_DEVICE, "%s: current device %d, but the graph lives on device %d", fn, cur, g->device);
+    return AG_OK;
+}
+
 int check_device_ptr(const void *p, int device, const char *name) {
     cudaPointerAttributes attr;
     cudaError_t err = cudaPointerGetAttributes(&attr, p);

@@ -216,6 +216,7 @@ int check_common(const ag_graph *g, int64_t H, int dtype, const void *scratch, s
     if (!g) return fail(AG_ERR_INVALID_ARG, "%s: null graph", fn);
     if (H < 1 || H > (int64_t(1) << 24)) return fail(AG_ERR_SHAPE, "%s: H = %lld outside [1, 2^24]", fn, (long long)H);
     if (dtype != AG_F32 && dtype != AG_BF16) return fail(AG_ERR_DTYPE, "%s: unknown dtype %d", fn, dtype);
+    if (int rc = check_current_device(g, fn)) return rc;
     *L = attn_layout(g, H);
     if (!scratch || scratch_bytes < L->total)
         return fail(AG_ERR_WORKSPACE, "%s: scratch of %zu bytes, need %zu", fn, scratch_bytes, L->total);

@@ -83,6 +83,8 @@ void clear_error();
 
 // AG_OK if p is device (or managed) memory usable on `device`.
 int check_device_ptr(const void *p, int device, const char *name);
+// AG_OK if the calling thread's current device is the graph's device.
+int check_current_device(const ag_graph *g, const char *fn);
 
 // Lowering-time workspace layout (shared by the size query and the lowering).
 struct Layout {

@@ -29,6 +29,8 @@
  *     name ends in _host.  The caller owns every buffer; the library never
  *     allocates device memory.  Pointers must stay valid until the work on
  *     `stream` has finished.
+ *   - Per-call functions run on the calling thread's current device, which
+ *     must be the device the graph was lowered on (AG_ERR_DEVICE otherwise).
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).  Per-call functions only enqueue work and return; results are
  *     ready when the stream reaches that point.
