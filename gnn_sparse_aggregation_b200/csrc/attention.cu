@@ -12,7 +12,7 @@
 // in one walk); the row statistics m_r (maximum)
 // and l_r (sum of exp(s - m_r)) come from one segmented reduction over the
 // forward CSR, walked in the same edge-balanced tiles as the SpMM: one warp
-// per tile, a Hillis-Steele segmented scan per 32 positions, rows cut by a
+// per tile, Hillis-Steele segmented scans per 32 positions, rows cut by a
 // tile boundary finished by a fixup pass in tile order.  Every reduction tree
 // is fixed by the positions alone, so results are deterministic.
 #include <cuda_runtime.h>
@@ -64,18 +64,34 @@ __device__ __forceinline__ float2 shfl2(float2 v, int src) {
     return make_float2(__shfl_sync(kFull, v.x, src), __shfl_sync(kFull, v.y, src));
 }
 
-// kSoftmaxStats: leaf (scale * a_e, 1); kSum: leaf (a_e * b_e, 0)
+// Leaf value of COO edge e: kSoftmaxStats the score scale * a_e, kSum a_e * b_e.
 template <int OP>
-__device__ __forceinline__ float2 leaf(const ReduceParams &P, int64_t p) {
-    const int e = __ldcs(P.order + p);
-    if (OP == kSoftmaxStats) return make_float2(P.scale * P.a[e], 1.f);
-    return make_float2(P.a[e] * P.b[e], 0.f);
+__device__ __forceinline__ float leaf_value(const ReduceParams &P, int e) {
+    return OP == kSoftmaxStats ? P.scale * P.a[e] : P.a[e] * P.b[e];
 }
 
-// One warp per tile of T consecutive forward-CSR positions.  The open row
-// (nz index `cur`) holds the running aggregate `acc`; within each chunk of 32
-// positions the row starts form a lane mask and a segmented inclusive scan
-// gives every segment's aggregate at its last lane.
+// Segmented inclusive scan over the 32 lanes (segment of lane i: from its
+// head hs to i): op is max or sum; hs = -1 for the segment that continues
+// the open row.
+template <bool MAX>
+__device__ __forceinline__ float seg_scan(float v, int lane, int hs) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(kFull, v, off);
+        if (lane >= off && lane - off >= hs) v = MAX ? fmaxf(v, o) : v + o;
+    }
+    return v;
+}
+
+// One warp per tile of T consecutive forward-CSR positions.  All leaves of
+// the tile are loaded first (the order map, then the gathered values, two
+// round trips per tile).  Within each chunk of 32 positions the row starts
+// form a lane mask; kSoftmaxStats takes a segmented maximum M per segment,
+// one exp(s - M) per lane and a segmented sum, so every segment's (M, l)
+// sits at its last lane; kSum takes one segmented sum.  The open row (nz
+// index `cur`) carries its aggregate `acc` across chunks.
+constexpr int kMaxChunks = kMaxTileEdges / 32;
+
 template <int OP>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const ReduceParams P) {
     const int64_t t = (int64_t(blockIdx.x) * kWarpsPerBlock) + (threadIdx.x >> 5);
@@ -83,13 +99,21 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const Reduce
     if (t >= P.n_tiles) return;  // whole warps
     const int64_t p0 = t * P.T;
     const int len = int(P.E - p0 < P.T ? P.E - p0 : P.T);
+    float x[kMaxChunks];
+    int e[kMaxChunks];
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) e[c] = c * 32 + lane < len ? __ldcs(P.order + p0 + c * 32 + lane) : -1;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) x[c] = e[c] >= 0 ? leaf_value<OP>(P, e[c]) : 0.f;
     int64_t cur = P.tile_nz[t];
     bool before = P.nz_rowptr[cur] < p0;
     float2 acc = identity<OP>();
-    for (int base = 0; base < len; base += 32) {
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+        const int base = c * 32;
+        if (base >= len) break;  // warp-uniform
         const int64_t cb = p0 + base;
         const int n = len - base < 32 ? len - base : 32;
-        float2 v = lane < n ? leaf<OP>(P, cb + lane) : identity<OP>();
         // starts of the rows after the open one that fall inside the chunk
         unsigned bit = 0;
         const int64_t k = cur + 1 + lane;
@@ -100,12 +124,16 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const Reduce
         const unsigned mask = __reduce_or_sync(kFull, bit);
         const unsigned upto = mask & (kFull >> (31 - lane));  // heads at lanes <= this one
         const int hs = upto ? 31 - __clz(upto) : -1;          // this lane's segment head
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            float2 o;
-            o.x = __shfl_up_sync(kFull, v.x, off);
-            o.y = __shfl_up_sync(kFull, v.y, off);
-            if (lane >= off && lane - off >= hs) v = combine<OP>(o, v);
+        const unsigned after = mask & ~(kFull >> (31 - lane)); // heads after this lane
+        const int se = after ? __ffs(after) - 2 : n - 1;      // last lane of this lane's segment
+        float2 v;
+        if (OP == kSoftmaxStats) {
+            const float s = lane < n ? x[c] : -INFINITY;
+            const float M = __shfl_sync(kFull, seg_scan<true>(s, lane, hs), se);
+            const float l = seg_scan<false>(lane < n ? expf(s - M) : 0.f, lane, hs);
+            v = make_float2(M, l);
+        } else {
+            v = make_float2(seg_scan<false>(lane < n ? x[c] : 0.f, lane, hs), 0.f);
         }
         const int nh = __popc(mask);
         if (nh > 0) {
