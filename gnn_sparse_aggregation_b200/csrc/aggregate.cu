@@ -991,12 +991,31 @@ k_bucket_staged(const float *__restrict__ in, const int32_t *__restrict__ slot,
     // all global loads of the chunk first (independent), then the staging
     int sl[kStageItems];
     float v[kStageItems];
+    float cnt[SCALED ? kStageItems : 1];  // in-degree of each item's destination
 #pragma unroll
     for (int k = 0; k < kStageItems; ++k) {
         const int i = k * kThreads + threadIdx.x;
         sl[k] = i < n ? __ldcs(slot + c0 + i) : -1;
         v[k] = (TO_BUCKETS && i < n) ? (in ? __ldcs(in + c0 + i) : 1.f) : 0.f;
-        if (TO_BUCKETS && SCALED && i < n) v[k] = per_dst(v[k], sc, c0 + i);
+    }
+    if constexpr (SCALED) {
+        // destinations of all items, then their row lengths: two waves of
+        // independent loads rather than a dependent pair per item
+        int d[kStageItems];
+#pragma unroll
+        for (int k = 0; k < kStageItems; ++k) {
+            const int i = k * kThreads + threadIdx.x;
+            d[k] = i < n ? __ldcs(sc.dst + c0 + i) : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < kStageItems; ++k) {
+            const int i = k * kThreads + threadIdx.x;
+            cnt[k] = i < n ? float(sc.rowptr[d[k] + 1] - sc.rowptr[d[k]]) : 1.f;  // >= 1: the edge itself
+        }
+        if (TO_BUCKETS) {
+#pragma unroll
+            for (int k = 0; k < kStageItems; ++k) v[k] = __fdiv_rn(v[k], cnt[k]);
+        }
     }
     int pos[kStageItems];
 #pragma unroll
@@ -1038,8 +1057,10 @@ k_bucket_staged(const float *__restrict__ in, const int32_t *__restrict__ slot,
 #pragma unroll
         for (int k = 0; k < kStageItems; ++k) {
             const int i = k * kThreads + threadIdx.x;
-            if (i < n && pos[k] >= 0)
-                __stcs(out + c0 + i, SCALED ? per_dst(stage_val[pos[k]], sc, c0 + i) : stage_val[pos[k]]);
+            if (i < n && pos[k] >= 0) {
+                if constexpr (SCALED) __stcs(out + c0 + i, __fdiv_rn(stage_val[pos[k]], cnt[k]));
+                else __stcs(out + c0 + i, stage_val[pos[k]]);
+            }
         }
     }
 }
@@ -1292,6 +1313,15 @@ int gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch, si
 }
 
 }  // namespace
+
+size_t spmm_scratch_edge_offset(const ag_graph *g, int64_t H, int which) {
+    const ScratchLayout L = scratch_layout(g, H);
+    return which == 0 ? L.w_b : L.dw_b;
+}
+void regroup_to_buckets(const ag_graph *g, int d, const float *in, float *out_b, cudaStream_t st) {
+    regroup(true, g->dir[d], in, g->E, out_b, st);
+}
+
 }  // namespace ag
 
 using namespace ag;

@@ -9,7 +9,8 @@
 //
 // The scores and the SpMMs run through this library's own entry points
 // (ag_sddmm_dw, ag_spmm_fwd, ag_spmm_dx, and ag_backward for dV with dalpha
-// in one walk); the row statistics m_r (maximum)
+// in one walk); the per-edge inputs of the row reductions are first regrouped
+// into the forward walk's window-bucketed order; the row statistics m_r (maximum)
 // and l_r (sum of exp(s - m_r)) come from one segmented reduction over the
 // forward CSR, walked in the same edge-balanced tiles as the SpMM: one warp
 // per tile, Hillis-Steele segmented scans per 32 positions, rows cut by a
@@ -49,8 +50,8 @@ __device__ __forceinline__ float2 identity() {
 }
 
 struct ReduceParams {
-    const int32_t *order;      // forward CSR position -> COO ordinal
-    const float *a;            // COO-order inputs
+    const int32_t *order;      // forward CSR position -> slot of its edge in `a` and `b`
+    const float *a;            // per-edge inputs, in the forward walk's window-bucketed order
     const float *b;
     float scale;
     int T;                     // positions per tile
@@ -211,14 +212,17 @@ AttnLayout attn_layout(const ag_graph *g, int64_t H) {
     return L;
 }
 
+// a_b, b_b: per-edge inputs already regrouped into the forward walk's
+// window-bucketed order, so that the walk's reads stay inside L2-sized
+// windows instead of one random sector per edge.
 template <int OP>
-int row_reduce(const ag_graph *g, const float *a, const float *b, float scale, float2 *partial, float2 *out,
+int row_reduce(const ag_graph *g, const float *a_b, const float *b_b, float scale, float2 *partial, float2 *out,
                cudaStream_t st) {
     const Direction &D = g->dir[0];
     ReduceParams P;
-    P.order = D.order;
-    P.a = a;
-    P.b = b;
+    P.order = D.bucket_of_pos;
+    P.a = a_b;
+    P.b = b_b;
     P.scale = scale;
     P.T = g->tile_edges;
     P.E = g->E;
@@ -281,7 +285,11 @@ int ag_attn_fwd(const ag_graph *g, const void *Q, const void *K, const void *V, 
         // raw scores dot(K[src], Q[dst]) in COO order, into alpha
         if ((rc = ag_sddmm_dw(g, K, Q, alpha, H, dtype, scr + L.spmm, spmm_bytes, stream)) != AG_OK) return rc;
         float2 *ml = reinterpret_cast<float2 *>(scr + L.rows);
-        rc = row_reduce<kSoftmaxStats>(g, alpha, nullptr, scale, reinterpret_cast<float2 *>(scr + L.partial), ml, st);
+        // the raw scores in the forward walk's bucket order (the SpMM scratch's
+        // per-edge array is free until the aggregation below)
+        float *s_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 0));
+        regroup_to_buckets(g, 0, alpha, s_b, st);
+        rc = row_reduce<kSoftmaxStats>(g, s_b, nullptr, scale, reinterpret_cast<float2 *>(scr + L.partial), ml, st);
         if (rc != AG_OK) return rc;
         k_softmax_alpha<<<flat_blocks(g->E), 256, 0, st>>>(alpha, g->coo_dst, ml, scale, g->E);
         cudaError_t err = cudaGetLastError();
@@ -312,9 +320,14 @@ int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, const void
         // dV = A_alpha^T dY and dalpha_e = dot(V[src], dY[dst]) in one transpose
         // walk (the weighted-sum backward with weights alpha and "features" V)
         if ((rc = ag_backward(g, alpha, V, dY, dV, ds, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
-        // c_r = sum over r's edges of alpha dalpha
+        // c_r = sum over r's edges of alpha dalpha, from bucket-ordered copies
+        // (the SpMM scratch's two per-edge arrays are free between the walks)
         float2 *c = reinterpret_cast<float2 *>(scr + L.rows);
-        rc = row_reduce<kSum>(g, alpha, ds, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
+        float *a_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 0));
+        float *d_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 1));
+        regroup_to_buckets(g, 0, alpha, a_b, st);
+        regroup_to_buckets(g, 0, ds, d_b, st);
+        rc = row_reduce<kSum>(g, a_b, d_b, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
         if (rc != AG_OK) return rc;
         k_attn_ds<<<flat_blocks(g->E), 256, 0, st>>>(alpha, ds, g->coo_dst, c, scale, g->E);
         cudaError_t err = cudaGetLastError();

@@ -101,4 +101,12 @@ inline bool staged_regroup(int64_t E) { return E > 0 && n_windows(E) <= kStageMa
 int pick_tile_edges(int64_t E);
 inline int64_t n_tiles_for(int64_t E, int T) { return (E + T - 1) / T; }
 
+// Shared with the attention kernels (defined in aggregate.cu).
+// Byte offsets, inside the per-call SpMM scratch of width H, of its two
+// per-edge float arrays (after the partial rows of rows cut by tiles).
+size_t spmm_scratch_edge_offset(const ag_graph *g, int64_t H, int which);
+// out_b[bucket slot of COO edge e] = in[e] for the walk direction d: COO
+// order into the window-bucketed order the walks read through bucket_of_pos.
+void regroup_to_buckets(const ag_graph *g, int d, const float *in, float *out_b, cudaStream_t st);
+
 }  // namespace ag
