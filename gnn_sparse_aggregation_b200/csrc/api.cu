@@ -1,6 +1,6 @@
 // api.cu -- status handling, pointer checks, workspace layout and handle
-// accessors of libaggraph.  The lowering lives in lower.cu and the per-call
-// kernels in aggregate.cu.
+// accessors of libaggraph.  The lowering lives in lower.cu, the per-call
+// kernels in aggregate.cu and attention.cu.
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>

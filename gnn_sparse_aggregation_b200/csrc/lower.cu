@@ -18,7 +18,11 @@
 //   4. the tile schedule of the per-call kernels: the non-empty rows
 //      compacted (ids and first positions), the empty rows listed, the row
 //      holding the first position of every tile, and the rows cut by a tile
-//      boundary (long ones first).
+//      boundary (long ones first);
+//   5. the weight windows: every edge's slot in an order grouped by windows
+//      of 2^20 consecutive CSR positions (COO order inside a window), the
+//      slot read at every CSR position, and the per-chunk staging table that
+//      lets the per-call regrouping write whole runs of slots.
 #include <climits>
 #include <cstdio>
 

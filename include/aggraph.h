@@ -116,8 +116,11 @@ AG_API size_t ag_graph_workspace_bytes(int64_t N, int64_t E);
  *   rowptr_f[N+1], col_f[E] = src[edge_order], edge_order[E]     (by destination)
  *   rowptr_t[N+1], col_t[E] = dst[transpose_order], transpose_order[E] (by source)
  * where each order map sends a CSR position to its COO ordinal, sorted by the
- * owner key with ties in ascending COO ordinal (a stable sort), plus the
- * degree-ordered row schedules used by the per-call kernels.
+ * owner key with ties in ascending COO ordinal (a stable sort), plus what
+ * the per-call kernels walk: the edge-balanced tile schedule of each CSR
+ * (rows with edges, the row holding each tile's first position, the rows cut
+ * by tile boundaries) and the tables that regroup per-edge arrays into
+ * windows of 2^20 consecutive CSR positions.
  *
  * Errors: AG_ERR_SHAPE for N < 1, E < 0, N or E >= 2^31; AG_ERR_INVALID_ARG
  * for null out/workspace or null src/dst with E > 0; AG_ERR_WORKSPACE if the
