@@ -63,7 +63,11 @@ constexpr int kMinBlocks = 4;  // resident CTAs per SM the register path is comp
 constexpr int kRingDepth = AG_RING_DEPTH;
 constexpr int kChunk = AG_CHUNK;
 
-enum Mode { kSpmm = 1, kSddmm = 2, kBoth = 3 };  // kBoth: feature and weight gradient in one walk
+// kBoth: feature and weight gradient in one walk.  Mean flags (ring walks
+// only): kRowScale multiplies every finished output row by inv_cnt[row]
+// (forward mean); kEdgeScale multiplies every edge's weight and dot product
+// by inv_cnt of its gathered column (the destination, in the transpose walk).
+enum Mode { kSpmm = 1, kSddmm = 2, kBoth = 3, kRowScale = 4, kEdgeScale = 8 };
 
 // A weight looked up through the bucketed layout: each 128-byte line of a
 // window is used by about 32 positions of that window's tiles, so it is kept
@@ -118,6 +122,7 @@ struct Params {
     void *out;                 // SpMM output [N, H]
     float *partial;            // [2 * n_tiles, H]: slot 2t = row continued from tile t-1, 2t+1 = row continued in tile t+1
     float *dw;                 // SDDMM output, COO order
+    const float *inv_cnt;      // mean modes: 1 / in-degree per node (forward CSR row lengths)
     int64_t E, H, n_nz;
     int64_t n_tiles;           // lane groups [0, n_tiles) walk one tile each
     int64_t n_zero;            // lane groups [n_tiles, n_tiles + n_zero) zero one empty row each
@@ -490,7 +495,10 @@ k_tiles_ring(const Params P) {
     float w_cur = 0.f, w_nxt = 0.f;
     if (gl < len) { c_cur = __ldcs(P.col + p0 + gl); e_cur = __ldcs(P.order + p0 + gl); }
     if (G + gl < len) { c_nxt = __ldcs(P.col + p0 + G + gl); e_nxt = __ldcs(P.order + p0 + G + gl); }
-    if ((MODE & kSpmm) && gl < len) w_cur = load_w(P.w + e_cur);
+    if ((MODE & kSpmm) && gl < len) {
+        w_cur = load_w(P.w + e_cur);
+        if constexpr ((MODE & kEdgeScale) != 0) w_cur *= P.inv_cnt[c_cur];
+    }
 
     const uint32_t row_bytes = uint32_t(H) * sizeof(T);
     auto issue = [&](int slot, int src) {
@@ -528,8 +536,18 @@ k_tiles_ring(const Params P) {
     auto write_open_row = [&](float *slot) {
         float o[NV][VEC];
         acc.get(o);
-        if (slot) store_slot<VEC, NV>(slot, 0, G, colok, o);
-        else store_row<T, VEC, NV>(out + int64_t(row) * H, 0, G, colok, o);
+        if (slot) {
+            store_slot<VEC, NV>(slot, 0, G, colok, o);
+        } else {
+            if constexpr ((MODE & kRowScale) != 0) {
+                const float r = P.inv_cnt[row];
+#pragma unroll
+                for (int k = 0; k < NV; ++k)
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) o[k][v] *= r;
+            }
+            store_row<T, VEC, NV>(out + int64_t(row) * H, 0, G, colok, o);
+        }
     };
     // the current row ended at the current position: write it, open the next
     // (runs only in the lane groups whose row ended: group-mask shuffles)
@@ -596,7 +614,7 @@ k_tiles_ring(const Params P) {
     // the unguarded batch of the gradient walks runs in chunks of U positions
     // (rolled), so that their longer row-switch code is inlined U times rather
     // than G times; the forward walk keeps the whole batch unrolled
-    constexpr int U = MODE == kSpmm ? G : chunk_of(G, D);
+    constexpr int U = (MODE & kSddmm) ? chunk_of(G, D) : G;
     static_assert(U % STEP == 0 && (U == G || (G - D) % U == 0) && (U >= D ? U % D == 0 : D % U == 0),
                   "chunk shape");
 
@@ -607,6 +625,8 @@ k_tiles_ring(const Params P) {
         }
         // weights of the next batch, indices of the one after
         if ((MODE & kSpmm)) w_nxt = (base + G + gl < len) ? load_w(P.w + e_nxt) : 0.f;
+        if constexpr ((MODE & kEdgeScale) != 0)
+            if (base + G + gl < len) w_nxt *= P.inv_cnt[c_nxt];
         c_nn = 0;
         e_nn = 0;
         if (base + 2 * G + gl < len) {
@@ -633,7 +653,8 @@ k_tiles_ring(const Params P) {
                 }
                 if ((MODE & kSddmm)) {
                     const float d = reduce_chunk<U, G>(dots, gl, FULL);
-                    if ((gl & ~(U - 1)) == j0) P.dw[e_cur] = d;  // lane j0 + t: position j0 + t
+                    if ((gl & ~(U - 1)) == j0)  // lane j0 + t: position j0 + t
+                        P.dw[e_cur] = (MODE & kEdgeScale) ? d * P.inv_cnt[c_cur] : d;
                 }
             }
         } else {
@@ -644,7 +665,7 @@ k_tiles_ring(const Params P) {
                 if ((MODE & kSddmm)) {
 #pragma unroll
                     for (int o = G / 2; o > 0; o >>= 1) d += __shfl_xor_sync(FULL, d, o, G);
-                    if (gl == j && base + j < len) P.dw[e_cur] = d;
+                    if (gl == j && base + j < len) P.dw[e_cur] = (MODE & kEdgeScale) ? d * P.inv_cnt[c_cur] : d;
                 }
                 refill(base, j, j % D, j + D < G ? c_cur : c_nxt, true);
             }
@@ -656,6 +677,14 @@ k_tiles_ring(const Params P) {
         else write_open_row(nullptr);
     }
     cp_async_wait<0>();
+}
+
+template <int VEC, int NV>
+__device__ __forceinline__ void scale_rows(float (&acc)[NV][VEC], float r) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[k][v] *= r;
 }
 
 // Rows cut by tile boundaries: out[row] = slot(2 * first + 1) + sum over the
@@ -670,7 +699,7 @@ constexpr int kStripes = 8;
 template <typename T, int VEC, int NV>
 __global__ void __launch_bounds__(kThreads)
 k_fixup(const int4 *__restrict__ spans, int64_t n_long, int64_t n_span, const float *__restrict__ partial,
-        void *out, int64_t H, int G, int log2G, int col_tiles) {
+        void *out, int64_t H, int G, int log2G, int col_tiles, const float *__restrict__ row_scale) {
     __shared__ float red[kStripes * 32 * NV * VEC];
     const int gl = threadIdx.x & (G - 1);
     const int gi = threadIdx.x >> log2G;
@@ -714,6 +743,7 @@ k_fixup(const int4 *__restrict__ spans, int64_t n_long, int64_t n_span, const fl
 #pragma unroll
                         for (int v = 0; v < VEC; ++v) acc[k][v] += red[(q * G * NV + k * G + gl) * VEC + v];
                 T *row = static_cast<T *>(out) + int64_t(sp.x) * H;
+                if (row_scale) scale_rows<VEC, NV>(acc, row_scale[sp.x]);
                 store_row<T, VEC, NV>(row, vbase, G, ok, acc);
             }
             __syncthreads();
@@ -743,6 +773,7 @@ k_fixup(const int4 *__restrict__ spans, int64_t n_long, int64_t n_span, const fl
             for (int k = 0; k < NV; ++k)
                 if (ok[k]) add_partial<VEC>(s1 + (vbase + int64_t(k) * G) * VEC, acc[k]);
         }
+        if (row_scale) scale_rows<VEC, NV>(acc, row_scale[sp.x]);
         store_row<T, VEC, NV>(static_cast<T *>(out) + int64_t(sp.x) * H, vbase, G, ok, acc);
     }
 }
@@ -828,7 +859,7 @@ void launch_main(const Params &P, const Shape &s, cudaStream_t st) {
             }
         }
     }
-    if constexpr (MODE != kBoth) {
+    if constexpr (MODE != kBoth && (MODE & (kRowScale | kEdgeScale)) == 0) {
         if (s.col_tiles == 1) k_tiles<T, VEC, NV, MODE, true><<<grid, kThreads, 0, st>>>(P);
         else k_tiles<T, VEC, NV, MODE, false><<<grid, kThreads, 0, st>>>(P);
     }
@@ -836,12 +867,12 @@ void launch_main(const Params &P, const Shape &s, cudaStream_t st) {
 
 template <typename T, int VEC, int NV>
 void launch_fixup(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s,
-                  cudaStream_t st) {
+                  const float *row_scale, cudaStream_t st) {
     const int64_t groups_per_block = kThreads / s.G;
     const int64_t short_spans = D.n_span - D.n_span_long;
     const unsigned grid = unsigned(D.n_span_long + (short_spans + groups_per_block - 1) / groups_per_block);
     k_fixup<T, VEC, NV><<<grid, kThreads, 0, st>>>(D.spans, D.n_span_long, D.n_span, partial, out, H, s.G,
-                                                   s.log2G, s.col_tiles);
+                                                   s.log2G, s.col_tiles, row_scale);
 }
 
 template <int MODE, typename T, int VEC>
@@ -866,23 +897,25 @@ void dispatch_main(const Params &P, const Shape &s, int dtype, cudaStream_t st) 
 }
 
 template <typename T, int VEC>
-void fixup_nv(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s, cudaStream_t st) {
+void fixup_nv(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s,
+              const float *row_scale, cudaStream_t st) {
     switch (s.nv) {
-        case 1: launch_fixup<T, VEC, 1>(D, partial, out, H, s, st); break;
-        case 2: launch_fixup<T, VEC, 2>(D, partial, out, H, s, st); break;
-        default: launch_fixup<T, VEC, 4>(D, partial, out, H, s, st); break;
+        case 1: launch_fixup<T, VEC, 1>(D, partial, out, H, s, row_scale, st); break;
+        case 2: launch_fixup<T, VEC, 2>(D, partial, out, H, s, row_scale, st); break;
+        default: launch_fixup<T, VEC, 4>(D, partial, out, H, s, row_scale, st); break;
     }
 }
 
+// row_scale: non-null multiplies every finished row by row_scale[row] (mean)
 void dispatch_fixup(const ag::Direction &D, const float *partial, void *out, int64_t H, const Shape &s,
-                    int dtype, cudaStream_t st) {
+                    int dtype, cudaStream_t st, const float *row_scale = nullptr) {
     if (dtype == AG_F32) {
-        if (s.vec == 4) fixup_nv<float, 4>(D, partial, out, H, s, st);
-        else fixup_nv<float, 1>(D, partial, out, H, s, st);
+        if (s.vec == 4) fixup_nv<float, 4>(D, partial, out, H, s, row_scale, st);
+        else fixup_nv<float, 1>(D, partial, out, H, s, row_scale, st);
     } else {
-        if (s.vec == 8) fixup_nv<bf16_t, 8>(D, partial, out, H, s, st);
-        else if (s.vec == 2) fixup_nv<bf16_t, 2>(D, partial, out, H, s, st);
-        else fixup_nv<bf16_t, 1>(D, partial, out, H, s, st);
+        if (s.vec == 8) fixup_nv<bf16_t, 8>(D, partial, out, H, s, row_scale, st);
+        else if (s.vec == 2) fixup_nv<bf16_t, 2>(D, partial, out, H, s, row_scale, st);
+        else fixup_nv<bf16_t, 1>(D, partial, out, H, s, row_scale, st);
     }
 }
 
@@ -915,7 +948,7 @@ int check_call(const ag_graph *g, int64_t H, int dtype, const char *fn) {
 
 // Per-call scratch: [partial rows][weights, bucketed][weight gradient, bucketed]
 struct ScratchLayout {
-    size_t partial, w_b, dw_b, total;
+    size_t partial, w_b, dw_b, inv, total;
 };
 ScratchLayout scratch_layout(const ag_graph *g, int64_t H) {
     ScratchLayout L;
@@ -925,7 +958,8 @@ ScratchLayout scratch_layout(const ag_graph *g, int64_t H) {
     L.partial = 0;
     L.w_b = align_up(part);
     L.dw_b = L.w_b + align_up(ev);
-    L.total = g->E > 0 ? L.dw_b + align_up(ev) : L.w_b;
+    L.inv = L.dw_b + align_up(ev);  // mean: 1 / in-degree per node
+    L.total = g->E > 0 ? L.inv + align_up(size_t(g->N) * 4) : L.w_b;
     return L;
 }
 size_t scratch_needed(const ag_graph *g, int64_t H) {
@@ -1100,6 +1134,27 @@ int check_scratch(const ag_graph *g, size_t need, const void *scratch, size_t sc
 }
 
 // SpMM over direction d: out = A_w X (d = 0) or A_w^T dY (d = 1).
+// The shapes the shared-memory ring walks take (see launch_main).
+bool ring_shape(const Shape &s, int dtype, int64_t H) {
+    return s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8) &&
+           int64_t(s.G) * s.nv * s.vec == H;
+}
+
+// inv[i] = 1 / (number of edges into i), 0 for rows without edges
+__global__ void k_inv_counts(const int32_t *__restrict__ rowptr, int64_t N, float *__restrict__ inv) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < N; i += int64_t(gridDim.x) * blockDim.x) {
+        const int c = rowptr[i + 1] - rowptr[i];
+        inv[i] = c > 0 ? 1.f / float(c) : 0.f;
+    }
+}
+float *mean_inverses(const ag_graph *g, char *scr, const ScratchLayout &SL, cudaStream_t st) {
+    float *inv = reinterpret_cast<float *>(scr + SL.inv);
+    const int64_t b = (g->N + kThreads - 1) / kThreads;
+    k_inv_counts<<<unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b)), kThreads, 0, st>>>(g->dir[0].rowptr, g->N,
+                                                                                          inv);
+    return inv;
+}
+
 EdgeScale mean_scale(const ag_graph *g, bool mean) {
     EdgeScale sc;
     if (mean) {
@@ -1118,7 +1173,7 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     if (!F || !out || (g->E > 0 && !w && !mean)) return fail(AG_ERR_INVALID_ARG, "%s: null w, input or output", fn);
     const ag::Direction &D = g->dir[d];
     const ScratchLayout SL = scratch_layout(g, H);
-    const size_t need = g->E > 0 ? SL.w_b + align_up(size_t(g->E) * 4) : SL.w_b;
+    const size_t need = g->E > 0 ? (mean ? SL.total : SL.w_b + align_up(size_t(g->E) * 4)) : SL.w_b;
     if ((rc = check_scratch(g, need, scratch, scratch_bytes, fn)) != AG_OK) return rc;
     if (check_ptrs) {
         if ((rc = check_device_ptr(F, g->device, "input")) != AG_OK) return rc;
@@ -1134,14 +1189,23 @@ int spmm(const ag_graph *g, int d, const float *w, const void *F, void *out, int
     P.out = out;
     P.partial = reinterpret_cast<float *>(scr + SL.partial);
     P.n_zero = g->N - D.n_nz;
+    // mean on the ring shapes: the forward walk scales finished rows, the
+    // transpose walk scales each edge by its destination (other shapes divide
+    // the weights while regrouping them)
+    const bool ring_mean = mean && g->E > 0 && ring_shape(s, dtype, H);
+    if (ring_mean) P.inv_cnt = mean_inverses(g, scr, SL, st);
     if (g->E > 0) {
         float *w_b = reinterpret_cast<float *>(scr + SL.w_b);
-        regroup(true, D, w, g->E, w_b, st, mean_scale(g, mean));
+        regroup(true, D, w, g->E, w_b, st, mean_scale(g, mean && !ring_mean));
         P.w = w_b;
         P.order = D.bucket_of_pos;  // the kernels read w[order[p]]: here the bucketed slot
     }
-    if (P.n_tiles + P.n_zero > 0) dispatch_main<kSpmm>(P, s, dtype, st);
-    if (D.n_span > 0) dispatch_fixup(D, P.partial, out, H, s, dtype, st);
+    if (P.n_tiles + P.n_zero > 0) {
+        if (ring_mean && d == 0) dispatch_main<kSpmm | kRowScale>(P, s, dtype, st);
+        else if (ring_mean) dispatch_main<kSpmm | kEdgeScale>(P, s, dtype, st);
+        else dispatch_main<kSpmm>(P, s, dtype, st);
+    }
+    if (D.n_span > 0) dispatch_fixup(D, P.partial, out, H, s, dtype, st, ring_mean && d == 0 ? P.inv_cnt : nullptr);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
@@ -1206,9 +1270,7 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
     const ag::Direction &D = g->dir[1];
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape s = pick_shape(H, dtype, X, dY, dX);
-    const bool ring = s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8) &&
-                      int64_t(s.G) * s.nv * s.vec == H;
-    if (!ring || g->E == 0) {
+    if (!ring_shape(s, dtype, H) || g->E == 0) {
         // shapes without the single walk: the two separate passes
         if ((rc = spmm(g, 1, w, dY, dX, H, dtype, scratch, scratch_bytes, stream, fn, false, mean)) != AG_OK)
             return rc;
@@ -1217,9 +1279,11 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
     char *scr = static_cast<char *>(scratch);
     float *w_b = reinterpret_cast<float *>(scr + SL.w_b);
     float *dw_b = reinterpret_cast<float *>(scr + SL.dw_b);
-    const EdgeScale sc = mean_scale(g, mean);
-    regroup(true, D, w, g->E, w_b, st, sc);
+    // mean: each edge's weight and dot scaled by its destination inside the walk
+    const EdgeScale sc{};
     Params P = base_params(g, D, H, s);
+    if (mean) P.inv_cnt = mean_inverses(g, scr, SL, st);
+    regroup(true, D, w, g->E, w_b, st, sc);
     P.order = D.bucket_of_pos;
     P.w = w_b;
     P.F = dY;
@@ -1228,7 +1292,8 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
     P.dw = dw_b;
     P.partial = reinterpret_cast<float *>(scr + SL.partial);
     P.n_zero = g->N - D.n_nz;
-    dispatch_main<kBoth>(P, s, dtype, st);
+    if (mean) dispatch_main<kBoth | kEdgeScale>(P, s, dtype, st);
+    else dispatch_main<kBoth>(P, s, dtype, st);
     if (D.n_span > 0) dispatch_fixup(D, P.partial, dX, H, s, dtype, st);
     regroup(false, D, dw_b, g->E, dw, st, sc);
     cudaError_t err = cudaGetLastError();

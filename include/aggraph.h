@@ -146,7 +146,8 @@ AG_API int ag_graph_get_stats(const ag_graph *g, ag_graph_stats *out);
  * buffers that hold the weights and the weight gradient regrouped by windows
  * of 2^20 consecutive CSR positions (the weights stay in COO order in the
  * caller's arrays; the regrouping keeps each tile's weight lookups inside
- * one window).  O(E / tile_edges * H + E), never E x H.
+ * one window), plus one float [N] of reciprocal in-degrees for the mean.
+ * O(E / tile_edges * H + E + N), never E x H.
  */
 AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
 
@@ -218,8 +219,11 @@ AG_API int ag_backward(const ag_graph *g, const float *w, const void *X, const v
  * the semiring structure):
  *   Y[r] = (1 / cnt(r)) * sum over edges e into r of w_e X[src_e],
  * cnt(r) = number of edges into r (duplicates counted), Y[r] = 0 when
- * cnt(r) = 0.  Each edge's weight is divided by cnt(dst_e) in fp32 (IEEE
- * division) before the same walk as ag_spmm_fwd.
+ * cnt(r) = 0.  The walk is that of ag_spmm_fwd; on the widths its shared-
+ * memory ring serves (16-byte vectors, at most two per lane, one pass over
+ * the width) every finished fp32 row sum is multiplied by the fp32
+ * reciprocal of cnt(r), on the others each weight is divided by cnt(dst_e)
+ * (IEEE division) while the weights are regrouped.
  *
  *   w        device float [E], COO order, or NULL for unit weights
  *   other arguments and errors as ag_spmm_fwd (same scratch size)
@@ -229,7 +233,9 @@ AG_API int ag_mean_fwd(const ag_graph *g, const float *w, const void *X, void *Y
 
 /*
  * Gradients of ag_mean_fwd for the upstream gradient dY, in one transpose
- * walk like ag_backward:
+ * walk like ag_backward (each edge's weight and dot product scaled by the
+ * fp32 reciprocal of cnt(dst_e) inside the walk on the ring widths, divided
+ * by cnt(dst_e) while the per-edge arrays are regrouped on the others):
  *   dX[s] = sum over edges e out of s of (w_e / cnt(dst_e)) dY[dst_e]
  *   dw_e  = dot(X[src_e], dY[dst_e]) / cnt(dst_e)
  *

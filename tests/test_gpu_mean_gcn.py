@@ -1,10 +1,11 @@
 """Parity of the mean aggregation and the GCN-normalised weights (CUDA path
 through the C ABI) with the fp64 oracle.
 
-Mean: the CUDA path divides each edge weight by the in-degree of its
-destination in fp32 (IEEE division, relative error 2^-24) before the same
-walk as the weighted sum, so the weighted-sum tolerances apply unchanged to
-the degree-scaled bounds the oracle returns.  GCN weights: with unit weights
+Mean: the CUDA path scales by 1 / in-degree once per row (forward) or per
+edge (backward), either as a product with the fp32 reciprocal (two
+roundings, relative 2^-23) or as an IEEE division while regrouping (one,
+2^-24), around the weighted-sum walks, so the weighted-sum tolerances apply
+unchanged to the degree-scaled bounds the oracle returns.  GCN weights: with unit weights
 the degrees are exact integers and the result carries four fp32 roundings
 (sqrt, division, two products): relative 1e-6.  With weights, the degree is
 an fp32 sum over the row (the width-1 SpMM, error within 1e-5 of the sum of

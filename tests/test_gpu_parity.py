@@ -88,14 +88,15 @@ def test_config_bitwise_reproducible(config):
 
 def test_config_no_edge_feature_temporary(config):
     """No [E, H] carrier: the per-call scratch holds two fp32 rows per tile for
-    rows cut by tile boundaries and two float [E] buffers, far below E x H
-    (witness section: the largest intermediate is bounded by node state, edge
-    state or row pointers)."""
+    rows cut by tile boundaries, two float [E] buffers and one float [N],
+    far below E x H (witness section: the largest intermediate is bounded by
+    node state, edge state or row pointers)."""
     wl, g = config
     s = g.stats
     spans = s["spanning_rows_f"] + s["spanning_rows_t"]
     rnd = lambda b: (b + 255) // 256 * 256
-    assert g.scratch_bytes(wl.H) == rnd(2 * 4 * wl.H * s["tiles"] if spans else 0) + 2 * rnd(4 * wl.E)
+    assert g.scratch_bytes(wl.H) == (rnd(2 * 4 * wl.H * s["tiles"] if spans else 0) + 2 * rnd(4 * wl.E)
+                                     + rnd(4 * wl.N))
     assert g.scratch_bytes(wl.H) < wl.E * wl.H * 4 // 4
     assert g.workspace.numel() < 80 * (wl.N + wl.E) + (1 << 16)
 
