@@ -58,3 +58,45 @@ def test_reference_arm_other_ranks_exit_without_work():
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2"],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_reference_arm_prints_the_contract_line():
+    # the oracle on a small workload: one JSON line with the base contract's
+    # keys, the reference marker and the CPU-baseline / end-to-end objects
+    import json
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "uniform",
+                          "--steps", "2", "--warmup", "1", "--cpu-seconds", "0.2"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 1
+    assert d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert "N=1024, E=8192, H=16" in d["config"]["workload"]
+
+
+def test_algorithmic_bytes_and_launch_count():
+    sys.path.insert(0, ROOT)
+    import bench
+    N, E, H = 1 << 22, 1 << 26, 128
+    a = bench.algorithmic_bytes(N, E, H, 2)
+    # CSR + order map + weights + input rows once + output rows once
+    assert a["fwd"] == 4 * (N + 1) + 12 * E + 2 * N * H * 2
+    assert abs(a["fwd"] / 1e9 - 2.97) < 0.01 and abs(a["backward"] / 1e9 - 4.31) < 0.01
+    rows = bench.row_bytes(N, E, H, 2)
+    assert rows["mean_fwd"] == a["fwd"] and rows["mean_backward"] == a["backward"]
+
+    class W:
+        pass
+    wl = W()
+    wl.E, wl.N = E, N
+    st = {"spanning_rows_f": 5, "spanning_rows_t": 0}
+    assert bench.launches_per_step_of(st, wl) == 3 + 3
+    wl.E = 0
+    assert bench.launches_per_step_of(st, wl) == 2
