@@ -279,3 +279,31 @@ def test_attn_sampled_form_matches_full():
     assert (np.abs(o["dQ"]) <= o["absdQ"] + 1e-12).all()
     assert (np.abs(o["dK"]) <= o["absdK"] + 1e-12).all()
     assert (np.abs(o["dV"]) <= o["absdV"] + 1e-12).all()
+
+
+def test_ext_pins_catch_planted_mistakes():
+    """Plausible slips, planted by calling the oracle with its operands
+    exchanged (on the CPU), must fail the invariants above."""
+    rng = np.random.default_rng(31)
+    N, E, H = 23, 90, 4
+    src, dst, w, X, G = rand_graph(rng, N, E, H, positive=True)
+    # GCN normalised by out-degrees (source and destination exchanged):
+    # the sqrt-degree fixed point of the in-degree normalisation fails
+    s2 = np.concatenate([src, np.arange(N, dtype=np.int32)])
+    d2 = np.concatenate([dst, np.arange(N, dtype=np.int32)])
+    w2 = np.concatenate([w, np.ones(N, np.float32)])
+    d_in = np.bincount(d2, weights=w2.astype(np.float64), minlength=N)
+    wrong = oracle.gcn_norm(d2, s2, N, w2)                     # degrees taken at the sources
+    An = dense_A(N, s2, d2, wrong)
+    assert not np.allclose(An @ np.sqrt(d_in), np.sqrt(d_in), rtol=1e-6)
+    # mean divided by out-degree (source and destination exchanged in the count)
+    cnt_in = np.bincount(dst, minlength=N).astype(np.float64)
+    inv = np.divide(1.0, cnt_in, out=np.zeros(N), where=cnt_in > 0)
+    right = inv[:, None] * (dense_A(N, src, dst, w) @ X)
+    swapped = oracle.mean_dx(dst, src, N, w, X)                 # sums at destinations, counts at sources
+    assert not np.allclose(swapped, right, atol=1e-9)
+    # softmax taken over the edges out of a source instead of into a destination
+    _, a_wrong, _ = oracle.attn_fwd(dst, src, N, X, X, X, 0.5)
+    sums = np.bincount(dst, weights=a_wrong, minlength=N)
+    has = np.bincount(dst, minlength=N) > 0
+    assert not np.allclose(sums[has], 1.0)
