@@ -155,8 +155,8 @@ AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
  * Forward aggregation Y = A_w X ("Decision": the forward pass walks the CSR
  * whose rows belong to destinations; reading guide Step 3: the gather / message /
  * scatter triple is one SpMM when the message is a scalar multiple of the
- * source row, PyG GraphConv's edge_weight * x_j of section "Reference
- * contract").
+ * source row, which is what PyG's GraphConv sends when given edge weights,
+ * section "Reference contract").
  *
  *   w        device float [E], COO order (may be NULL when E == 0)
  *   X        device [N, H] of dtype
@@ -171,8 +171,8 @@ AG_API int ag_spmm_fwd(const ag_graph *g, const float *w, const void *X, void *Y
                 int dtype, void *scratch, size_t scratch_bytes, void *stream);
 
 /*
- * Feature gradient dX = A_w^T dY ("Decision": dX reuses the same CSR
- * traversal, here over the source-owned transpose CSR and transpose_order).
+ * Feature gradient dX = A_w^T dY ("Decision": the same kind of CSR walk,
+ * here over the source-owned transpose CSR and transpose_order).
  * Arguments and errors as ag_spmm_fwd, with dY in place of X and dX in place
  * of Y; rows without out-edges are 0.
  */
@@ -181,7 +181,8 @@ AG_API int ag_spmm_dx(const ag_graph *g, const float *w, const void *dY, void *d
 
 /*
  * Weight gradient dw_e = dot(X[src_e], dY[dst_e]) ("Edge order is explicit";
- * "Exact witness": one output per edge, reduced over the feature width only;
+ * "Exact witness": exactly one value per edge, a sum over the H feature
+ * positions;
  * reading guide Step 4: SDDMM, a dense product evaluated only at the
  * adjacency's nonzeros).
  *
