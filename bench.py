@@ -113,14 +113,40 @@ def launches_per_step_of(st, wl):
 STEP_SOURCES = ("aggregate.cu", "device_common.cuh", "internal.h", "lower.cu")
 
 
+def code_only(text):
+    """C/C++ source without comments, trailing blanks or empty lines: the part
+    of a file the compiler sees."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def source_hash():
-    """Hash of the sources of the step's kernels and of the schedule they walk
-    (a traffic record taken on other sources is not reported)."""
+    """Hash of the code (comments left out) of the step's kernels and of the
+    schedule they walk: a traffic record taken on other code is not reported."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gnn_sparse_aggregation_b200", "csrc")
     for fn in STEP_SOURCES:
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + f.read())
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+            h.update(fn.encode() + code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

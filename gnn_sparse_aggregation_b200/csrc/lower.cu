@@ -2,8 +2,9 @@
 //
 // tinymesh "Weighted aggregation experiment", section "Edge order is
 // explicit": connectivity is sorted by owner without detaching the weights.
-// Both order maps send a CSR position to the original COO ordinal, and
-// duplicate source-target pairs keep separate positions.  Section "Exact
+// edge_order and transpose_order take a slot of the sorted CSR back to the
+// edge's index in the caller's COO list; two edges with the same endpoints
+// are two slots, never merged.  Section "Exact
 // witness": edges 0->2, 1->2, 0->1 lower to edge_order = (2, 0, 1), i.e. ties
 // between edges of one owner stay in COO order (a stable sort on the owner).
 //

@@ -154,9 +154,9 @@ AG_API size_t ag_spmm_scratch_bytes(const ag_graph *g, int64_t H);
 /*
  * Forward aggregation Y = A_w X ("Decision": the forward pass walks the CSR
  * whose rows belong to destinations; reading guide Step 3: the gather / message /
- * scatter triple is one SpMM when the message is a scalar multiple of the
- * source row, which is what PyG's GraphConv sends when given edge weights,
- * section "Reference contract").
+ * scatter triple reduces to one SpMM whenever each message is just the
+ * source's feature row times a per-edge number, which is what PyG's GraphConv
+ * sends when given edge weights, section "Reference contract").
  *
  *   w        device float [E], COO order (may be NULL when E == 0)
  *   X        device [N, H] of dtype

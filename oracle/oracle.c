@@ -26,10 +26,10 @@
  * feature values convert to fp64 exactly, so every product and sum below is
  * done in fp64 on the exact input values.
  *
- * Lowering ("Edge order is explicit"): edge_order maps a forward-CSR position
- * to the original COO ordinal, sorted by destination; transpose_order does the
- * same for the transpose CSR, sorted by source.  Duplicate pairs keep separate
- * positions.  Within one owner row the order is ascending COO ordinal (a
+ * Lowering ("Edge order is explicit"): edge_order[p] is the COO index of the
+ * edge stored at slot p of the forward CSR (slots grouped by destination);
+ * transpose_order[p] is the same for the transpose CSR (grouped by source).
+ * Repeated (source, target) pairs occupy one slot each.  Within one owner row the order is ascending COO ordinal (a
  * stable sort on the owner key alone); this is the reading that reproduces the
  * printed witness edge_order = (2, 0, 1) of section "Exact witness".  The
  * stable sort is written out as a counting sort.

@@ -100,3 +100,12 @@ def test_algorithmic_bytes_and_launch_count():
     assert bench.launches_per_step_of(st, wl) == 3 + 3
     wl.E = 0
     assert bench.launches_per_step_of(st, wl) == 2
+
+
+def test_traffic_record_keys_on_code_not_comments():
+    sys.path.insert(0, ROOT)
+    import bench
+    src = 'int a = 1; // note\n/* block\n comment */ const char *s = "// kept /* too */";\n\n  char c = \'"\';  \n'
+    assert bench.code_only(src) == 'int a = 1;\n  const char *s = "// kept /* too */";\n  char c = \'"\';'
+    assert bench.code_only("x = 1;\n// only a comment\n") == bench.code_only("x = 1;\n")
+    assert bench.code_only("x = 1;") != bench.code_only("x = 2;")

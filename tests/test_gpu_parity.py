@@ -89,8 +89,8 @@ def test_config_bitwise_reproducible(config):
 def test_config_no_edge_feature_temporary(config):
     """No [E, H] carrier: the per-call scratch holds two fp32 rows per tile for
     rows cut by tile boundaries, two float [E] buffers and one float [N],
-    far below E x H (witness section: the largest intermediate is bounded by
-    node state, edge state or row pointers)."""
+    far below E x H (witness section: no buffer larger than the per-node,
+    per-edge or row-pointer arrays is allowed)."""
     wl, g = config
     s = g.stats
     spans = s["spanning_rows_f"] + s["spanning_rows_t"]

@@ -5,9 +5,9 @@ operand, a wrong index, a dropped term, a sign, an unstable sort) fails at
 least one test: the hand-derived "Exact witness" of the tinymesh "Weighted
 aggregation experiment" page, dense matrix products by brute force (numpy),
 library stable sorts, the adjoint identity, finite differences of the linear
-loss, and the page's edge cases (section "Exact witness": paired COO
-permutations, duplicate edges with different weights, isolated and empty rows,
-the one-node case).
+loss, and the edge cases listed in section "Exact witness" (two COO
+orderings of one graph, repeated edges carrying unequal weights, nodes with
+no edges, a graph of a single node).
 """
 import numpy as np
 import pytest
