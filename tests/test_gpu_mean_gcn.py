@@ -106,13 +106,14 @@ def test_mean_narrow_and_ragged_widths(agb, H, dtype):
     assert_within(dw, rw, bw, TOL_DW, f"H={H} mean dw")
 
 
-def test_mean_of_unit_in_degree_equals_weighted_sum(agb):
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_mean_of_unit_in_degree_equals_weighted_sum(agb, dtype):
     # every node receives exactly one edge: mean == sum, bit for bit
     N, H = 3000, 64
     rng = np.random.default_rng(3)
     src = rng.permutation(N)
     dst = np.arange(N)
-    wl = workloads.custom(N, src, dst, H, seed=5, device=DEV)
+    wl = workloads.custom(N, src, dst, H, seed=5, feature_dtype=dtype, device=DEV)
     g = agb.ag_graph_lower(wl.src, wl.dst, N)
     Y1 = agb.ag_mean_fwd(g, wl.w, wl.X)
     Y2 = agb.ag_spmm_fwd(g, wl.w, wl.X)

@@ -158,6 +158,33 @@ def test_unaligned_feature_pointers_take_the_narrow_path(agb, dtype):
     assert torch.equal(Y.float(), ref.float())
 
 
+def _rows_per_tile_graph(kind, rng):
+    N = 6000
+    if kind == "unit_rows":      # in-degree 1: a new row at every position
+        dst = rng.permutation(N)
+    elif kind == "short_rows":   # in-degree 1..3 with empty rows between
+        nodes = rng.choice(N, N // 2, replace=False)
+        dst = np.repeat(nodes, rng.integers(1, 4, nodes.size))
+    else:                        # one row cut by many tiles among rows of in-degree 1 and 9
+        dst = np.concatenate([np.full(30000, 17), np.arange(0, N, 3), np.repeat(np.arange(1, N, 7), 9)])
+    src = rng.integers(0, N, dst.size)
+    perm = rng.permutation(dst.size)
+    return N, src[perm].astype(np.int32), dst[perm].astype(np.int32)
+
+
+@pytest.mark.parametrize("H", [64, 128])
+@pytest.mark.parametrize("kind", ["unit_rows", "short_rows", "heavy_and_unit"])
+def test_rows_per_tile_extremes(agb, H, kind):
+    """bf16 rows of 64 and 128 features (the ring walks) on the extremes of
+    rows per tile: every row a single edge (a row switch at every position),
+    short rows with empty rows between them, and a row cut by many tiles among
+    one-edge rows."""
+    rng = np.random.default_rng(H + len(kind))
+    N, src, dst = _rows_per_tile_graph(kind, rng)
+    wl, g = graph(agb, N, src, dst, H, torch.bfloat16)
+    check_full(g, wl, f"{kind} H={H}")
+
+
 def test_empty_graph_and_one_node(agb):
     # E = 0: outputs are exact zeros, dw is empty
     wl, g = graph(agb, 9, [], [], 6)
