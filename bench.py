@@ -334,9 +334,9 @@ def our_arm(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    from gnn_sparse_aggregation_b200 import _build
+    from __graft_entry__ import build_library
     if rank == 0 or world == 1:
-        _build.build()
+        build_library()
     if world > 1:
         dist.barrier()
     import gnn_sparse_aggregation_b200 as agb
@@ -446,7 +446,9 @@ def our_arm(args):
         hY, hdX = torch.empty_like(hX).pin_memory(), torch.empty_like(hX).pin_memory()
         hdw = torch.empty_like(hw).pin_memory()
         staging = torch.empty(agb.ag_step_staging_bytes(g, wl.H, wl.X.dtype), dtype=torch.uint8, device=dev)
-        agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging)
+        # back-to-back steps through the pipelined entry point: each step's
+        # copies in overlap the previous step's copies out
+        agb.ag_step_host_pipelined(g, hw, hX, hdY, hY, hdX, hdw, staging)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
@@ -454,7 +456,7 @@ def our_arm(args):
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(Ke):
-            agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging)
+            agb.ag_step_host_pipelined(g, hw, hX, hdY, hY, hdX, hdw, staging)
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
@@ -462,7 +464,7 @@ def our_arm(args):
         e2e = {"value": whole_job_rate(world, wl.E * wl.H, Ke, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": hw.numel() * 4 + 2 * hX.numel() * elem,
                "d2h_bytes_per_step": 2 * hX.numel() * elem + hdw.numel() * 4,
-               "steps": Ke, "ms_per_step": e_ms / Ke}
+               "steps": Ke, "ms_per_step": e_ms / Ke, "api": "ag_step_host_pipelined"}
         del staging, hw, hX, hdY, hY, hdX, hdw
 
     hbm, peak_kind = peaks()

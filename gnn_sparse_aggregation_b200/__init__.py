@@ -15,6 +15,7 @@ and "Edge order is explicit"), with A_w[dst_e, src_e] = w_e:
     ag_sddmm_dw(g, X, dY)        -> dw_e = dot(X[src_e], dY[dst_e])   (COO order)
     ag_backward(g, w, X, dY)     -> (dX, dw) in one pass over the transpose CSR
     ag_step_host(g, w, X, dY, ...)  the three from host buffers, copies included
+    ag_step_host_pipelined(...)     the same for back-to-back steps (copies overlap across steps)
 """
 from __future__ import annotations
 
@@ -25,7 +26,7 @@ import re
 import torch
 
 __all__ = ["AggraphError", "Graph", "ag_graph_lower", "ag_spmm_fwd", "ag_spmm_dx", "ag_sddmm_dw", "ag_backward",
-           "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward", "ag_step_host", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
+           "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward", "ag_step_host", "ag_step_host_pipelined", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
            "declared_symbols", "AG_F32", "AG_BF16"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaggraph.so")
@@ -38,7 +39,7 @@ _STATUS = {0: "AG_OK", 1: "AG_ERR_INVALID_ARG", 2: "AG_ERR_SHAPE", 3: "AG_ERR_DT
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m gnn_sparse_aggregation_b200._build` "
+        f"{LIB_PATH} is missing: build it with `python gnn_sparse_aggregation_b200/_build.py` "
         "(or __graft_entry__.build()); there is no fallback implementation")
 
 
@@ -94,13 +95,14 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_step_staging_bytes.argtypes = [_P, _I64, _I]
     handle.ag_step_staging_bytes.restype = _SZ
     handle.ag_step_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_step_host_pipelined.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_graph_free.argtypes = [_P]
     handle.ag_graph_free.restype = None
     handle.ag_last_error.restype = ctypes.c_char_p
     handle.ag_status_string.argtypes = [_I]
     handle.ag_status_string.restype = ctypes.c_char_p
     for name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
-                 "ag_sddmm_dw", "ag_backward", "ag_spmm_fwd_static_scratch", "ag_step_host", "ag_abi_version",
+                 "ag_sddmm_dw", "ag_backward", "ag_spmm_fwd_static_scratch", "ag_step_host", "ag_step_host_pipelined", "ag_abi_version",
                  "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward"):
         getattr(handle, name).restype = _I
     return handle
@@ -447,18 +449,27 @@ def ag_step_staging_bytes(g: Graph, H: int, dtype: torch.dtype) -> int:
 
 
 def ag_step_host(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, Y: torch.Tensor,
-                 dX: torch.Tensor, dw: torch.Tensor, staging: torch.Tensor, stream=None) -> None:
+                 dX: torch.Tensor, dw: torch.Tensor, staging: torch.Tensor, stream=None, pipelined=False) -> None:
     """Forward, feature gradient and weight gradient from host buffers.
 
     w, X, dY are host inputs and Y, dX, dw host outputs (page-locked tensors
     make the copies asynchronous); staging is a device uint8 tensor of
     ag_step_staging_bytes(g, H, X.dtype) bytes.  Enqueues on `stream`; the
-    outputs are valid after that stream is synchronized."""
+    outputs are valid after that stream is synchronized.  pipelined=True calls
+    ag_step_host_pipelined (the staging tensor then belongs to the steps)."""
     for name, t in (("w", w), ("X", X), ("dY", dY), ("Y", Y), ("dX", dX), ("dw", dw)):
         if t.is_cuda or not t.is_contiguous():
             raise AggraphError(4, f"{name} must be a contiguous host tensor")
     code = _dtype_code(X)
     _need_cuda("staging", staging)
-    _check(lib.ag_step_host(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(Y), _ptr(dX), _ptr(dw),
-                            X.shape[1], code, ctypes.c_void_p(staging.data_ptr()), staging.numel(),
-                            _stream(g.device, stream)))
+    fn = lib.ag_step_host_pipelined if pipelined else lib.ag_step_host
+    _check(fn(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(Y), _ptr(dX), _ptr(dw),
+              X.shape[1], code, ctypes.c_void_p(staging.data_ptr()), staging.numel(),
+              _stream(g.device, stream)))
+
+
+def ag_step_host_pipelined(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, Y: torch.Tensor,
+                           dX: torch.Tensor, dw: torch.Tensor, staging: torch.Tensor, stream=None) -> None:
+    """ag_step_host for back-to-back steps: this step's copies in overlap the
+    previous step's copies out on the same staging tensor."""
+    ag_step_host(g, w, X, dY, Y, dX, dw, staging, stream, pipelined=True)

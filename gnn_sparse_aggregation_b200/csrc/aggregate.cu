@@ -1477,7 +1477,7 @@ int step_streams(int device, cudaStream_t *in, cudaStream_t *out) {
 // Events of one ag_step_host call, released when the call returns (the
 // runtime keeps them alive until the work that waits on them is done).
 struct StepEvents {
-    cudaEvent_t e[5] = {};
+    cudaEvent_t e[6] = {};
     cudaError_t create() {
         for (auto &x : e) {
             cudaError_t err = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
@@ -1490,6 +1490,54 @@ struct StepEvents {
             if (x) cudaEventDestroy(x);
     }
 };
+
+// Pipelined steps: per staging buffer, an event recorded after the last
+// read of its input part (w, X, dY) by a step's fused backward pass.  The
+// input copies of the next pipelined step on that buffer wait for this
+// event only, so they overlap the previous step's copies out.  A bounded
+// table: a buffer whose entry was reused, or that was never seen, gets the
+// full ordering after `stream` again.
+constexpr int kStagingSlots = 16;
+struct StagingOrder {
+    const void *staging = nullptr;
+    int device = -1;
+    cudaEvent_t done = nullptr;
+};
+StagingOrder g_staging[kStagingSlots];
+int g_staging_next = 0;
+
+StagingOrder *find_staging(const void *staging, int device) {
+    for (auto &s : g_staging)
+        if (s.done && s.staging == staging && s.device == device) return &s;
+    return nullptr;
+}
+
+// Make `in` wait for the previous step's reads of the staging buffer's
+// inputs (pipelined), or for everything on `st` so far (first use).
+cudaError_t staging_wait_inputs(const void *staging, int device, cudaStream_t st, cudaStream_t in, cudaEvent_t tmp) {
+    std::lock_guard<std::mutex> lock(g_step_mu);
+    if (StagingOrder *s = find_staging(staging, device)) return cudaStreamWaitEvent(in, s->done, 0);
+    StagingOrder &s = g_staging[g_staging_next];
+    g_staging_next = (g_staging_next + 1) % kStagingSlots;
+    if (s.done) cudaEventDestroy(s.done);  // released once its pending waits are done
+    s = StagingOrder{};
+    cudaError_t err = cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming);
+    if (err != cudaSuccess) {
+        s.done = nullptr;
+        return err;
+    }
+    s.staging = staging;
+    s.device = device;
+    err = cudaEventRecord(tmp, st);
+    return err == cudaSuccess ? cudaStreamWaitEvent(in, tmp, 0) : err;
+}
+
+// After a step's backward pass (on st): the staging buffer's inputs are read.
+cudaError_t staging_mark_read(const void *staging, int device, cudaStream_t st) {
+    std::lock_guard<std::mutex> lock(g_step_mu);
+    if (StagingOrder *s = find_staging(staging, device)) return cudaEventRecord(s->done, st);
+    return cudaSuccess;
+}
 }  // namespace
 
 extern "C" {
@@ -1515,19 +1563,22 @@ size_t ag_step_staging_bytes(const ag_graph *g, int64_t H, int dtype) {
     return total;
 }
 
-int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, const void *dY_host,
-                 void *Y_host, void *dX_host, float *dw_host, int64_t H, int dtype, void *staging,
-                 size_t staging_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+int step_host(const ag_graph *g, const float *w_host, const void *X_host, const void *dY_host, void *Y_host,
+              void *dX_host, float *dw_host, int64_t H, int dtype, void *staging, size_t staging_bytes,
+              void *stream, bool pipelined, const char *fn) {
     clear_error();
-    int rc = check_call(g, H, dtype, "ag_step_host");
+    int rc = check_call(g, H, dtype, fn);
     if (rc != AG_OK) return rc;
     if (!X_host || !dY_host || !Y_host || !dX_host || (g->E > 0 && (!w_host || !dw_host)) || !staging)
-        return fail(AG_ERR_INVALID_ARG, "ag_step_host: null buffer");
+        return fail(AG_ERR_INVALID_ARG, "%s: null buffer", fn);
     size_t off[7], total = 0;
     staging_layout(g, H, dtype, off, &total);
     if (staging_bytes < total)
-        return fail(AG_ERR_WORKSPACE, "ag_step_host: staging of %zu bytes, need %zu", staging_bytes, total);
-    if (!aligned(staging, kAlign)) return fail(AG_ERR_WORKSPACE, "ag_step_host: staging must be 256-byte aligned");
+        return fail(AG_ERR_WORKSPACE, "%s: staging of %zu bytes, need %zu", fn, staging_bytes, total);
+    if (!aligned(staging, kAlign)) return fail(AG_ERR_WORKSPACE, "%s: staging must be 256-byte aligned", fn);
     if ((rc = check_device_ptr(staging, g->device, "staging")) != AG_OK) return rc;
     char *base = static_cast<char *>(staging);
     float *w = reinterpret_cast<float *>(base + off[0]);
@@ -1551,23 +1602,33 @@ int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, con
         if (err == cudaSuccess) err = cudaStreamWaitEvent(s, e, 0);
     };
     const size_t scr = scratch_needed(g, H);  // staging's scratch part
-    // w and X first; dY follows on its own stream while the forward pass runs
-    copy(w, w_host, wb, cudaMemcpyHostToDevice, st);
-    copy(X, X_host, feat, cudaMemcpyHostToDevice, st);
-    record(ev.e[0], st);
-    wait(s_in, ev.e[0]);
+    if (pipelined) {
+        // all inputs on the helper stream, after the previous step's backward
+        // pass on this staging buffer (not after its copies out)
+        if (err == cudaSuccess) err = staging_wait_inputs(staging, g->device, st, s_in, ev.e[5]);
+        copy(w, w_host, wb, cudaMemcpyHostToDevice, s_in);
+        copy(X, X_host, feat, cudaMemcpyHostToDevice, s_in);
+        record(ev.e[0], s_in);
+        wait(st, ev.e[0]);
+    } else {
+        // w and X first; dY follows on its own stream while the forward pass runs
+        copy(w, w_host, wb, cudaMemcpyHostToDevice, st);
+        copy(X, X_host, feat, cudaMemcpyHostToDevice, st);
+        record(ev.e[0], st);
+        wait(s_in, ev.e[0]);
+    }
     copy(dY, dY_host, feat, cudaMemcpyHostToDevice, s_in);
     record(ev.e[1], s_in);
-    if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy in");
-    if ((rc = spmm(g, 0, w, X, Y, H, dtype, scratch, scr, stream, "ag_step_host", false)) != AG_OK) return rc;
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    if ((rc = spmm(g, 0, w, X, Y, H, dtype, scratch, scr, stream, fn, false)) != AG_OK) return rc;
     // Y goes out (device to host) while dY still comes in (host to device)
     record(ev.e[2], st);
     wait(s_out, ev.e[2]);
     copy(Y_host, Y, feat, cudaMemcpyDeviceToHost, s_out);
     wait(st, ev.e[1]);
-    if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy");
-    if ((rc = backward(g, w, X, dY, dX, dw, H, dtype, scratch, scr, stream, "ag_step_host", false)) != AG_OK)
-        return rc;
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    if ((rc = backward(g, w, X, dY, dX, dw, H, dtype, scratch, scr, stream, fn, false)) != AG_OK) return rc;
+    if (err == cudaSuccess) err = staging_mark_read(staging, g->device, st);
     record(ev.e[3], st);
     wait(s_out, ev.e[3]);
     copy(dX_host, dX, feat, cudaMemcpyDeviceToHost, s_out);
@@ -1575,10 +1636,26 @@ int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, con
     // `stream` covers every copy: the caller synchronizes it alone
     record(ev.e[4], s_out);
     wait(st, ev.e[4]);
-    if (err != cudaSuccess) return cuda_fail(err, "ag_step_host: copy out");
+    if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
 }
+}  // namespace
 
+extern "C" {
+
+int ag_step_host(const ag_graph *g, const float *w_host, const void *X_host, const void *dY_host,
+                 void *Y_host, void *dX_host, float *dw_host, int64_t H, int dtype, void *staging,
+                 size_t staging_bytes, void *stream) {
+    return step_host(g, w_host, X_host, dY_host, Y_host, dX_host, dw_host, H, dtype, staging, staging_bytes,
+                     stream, false, "ag_step_host");
+}
+
+int ag_step_host_pipelined(const ag_graph *g, const float *w_host, const void *X_host, const void *dY_host,
+                           void *Y_host, void *dX_host, float *dw_host, int64_t H, int dtype, void *staging,
+                           size_t staging_bytes, void *stream) {
+    return step_host(g, w_host, X_host, dY_host, Y_host, dX_host, dw_host, H, dtype, staging, staging_bytes,
+                     stream, true, "ag_step_host_pipelined");
+}
 
 // ---------------------------------------------------------------------------- forward without caller scratch
 

@@ -334,6 +334,26 @@ AG_API int ag_step_host(const ag_graph *g, const float *w_host, const void *X_ho
                  int64_t H, int dtype, void *staging, size_t staging_bytes, void *stream);
 
 /*
+ * ag_step_host for a sequence of steps (an interface addition of this
+ * library): the same arguments, copies and results, but this call's copies
+ * in (w, X, dY, all on the helper stream) are ordered only after the previous
+ * step's fused backward pass on the same staging buffer, not after that
+ * step's copies out.  Back-to-back steps on one staging buffer therefore
+ * bring the next step's inputs in while the previous step's dX and dw go out.
+ * `stream` is still ordered after every copy of this call.
+ *
+ * The staging buffer belongs to the steps between calls: no other work may
+ * read or write it.  The first call on a buffer (or on one of more than 16
+ * buffers in use) is ordered after everything on `stream`, like ag_step_host;
+ * an ag_step_host call on the same buffer keeps the order for the next
+ * pipelined call.  The host input buffers are read until `stream` has been
+ * synchronized after the call.
+ */
+AG_API int ag_step_host_pipelined(const ag_graph *g, const float *w_host, const void *X_host,
+                 const void *dY_host, void *Y_host, void *dX_host, float *dw_host,
+                 int64_t H, int dtype, void *staging, size_t staging_bytes, void *stream);
+
+/*
  * Forward aggregation without caller scratch (no counterpart on the pages:
  * an interface addition of this library).
  *

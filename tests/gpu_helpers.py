@@ -15,8 +15,8 @@ TOL_DW = 1e-5
 
 
 def lib():
-    from gnn_sparse_aggregation_b200 import _build
-    _build.build()
+    from __graft_entry__ import build_library
+    build_library()
     import gnn_sparse_aggregation_b200 as agb
     return agb
 

@@ -12,8 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def agb():
-    from gnn_sparse_aggregation_b200 import _build
-    _build.build()
+    from __graft_entry__ import build_library
+    build_library()
     import gnn_sparse_aggregation_b200 as m
     return m
 
@@ -79,6 +79,8 @@ def test_host_side_rejections_without_gpu(agb):
     assert lib.ag_graph_get_stats(None, None) == 1
     assert lib.ag_spmm_scratch_bytes(None, 4) == 0
     assert lib.ag_step_staging_bytes(None, 4, 0) == 0
+    for step in (lib.ag_step_host, lib.ag_step_host_pipelined):
+        assert step(None, None, None, None, None, None, None, 4, 0, None, 0, None) == 1
     lib.ag_graph_free(None)
 
 

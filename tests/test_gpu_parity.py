@@ -333,6 +333,36 @@ def test_step_from_host_buffers_orders_on_the_callers_stream(agb):
         assert torch.equal(hdw, dw)
 
 
+@pytest.mark.parametrize("modes", [(True, True, True, True, True), (True, False, True, True, False)])
+def test_pipelined_steps_keep_each_steps_results(agb, modes):
+    """Back-to-back pipelined steps (mixed with plain ones) on one staging
+    buffer and one side stream: each step's inputs come in while the previous
+    step's results go out, and every step must still return exactly its own
+    results.  Copies of a few MB each, so that the overlap is real."""
+    src, dst = workloads.rmat_edges(17, 16, seed=6)
+    N = 1 << 17
+    wl, g = graph(agb, N, src.numpy(), dst.numpy(), 64, torch.bfloat16)
+    staging = torch.empty(agb.ag_step_staging_bytes(g, wl.H, torch.bfloat16), dtype=torch.uint8, device=DEV)
+    ins, outs, refs = [], [], []
+    for k in range(len(modes)):
+        w = wl.w * (k + 1)
+        X = (wl.X.float() * (k + 1) - k).bfloat16()
+        dY = (wl.dY.float() + k).bfloat16()
+        refs.append(tuple(t.cpu() for t in (g.fwd(w, X), *g.backward(w, X, dY))))
+        ins.append(tuple(t.cpu().pin_memory() for t in (w, X, dY)))
+        outs.append((torch.empty_like(ins[-1][1]).pin_memory(), torch.empty_like(ins[-1][1]).pin_memory(),
+                     torch.empty_like(ins[-1][0]).pin_memory()))
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    for pipelined, (hw, hX, hdY), (hY, hdX, hdw) in zip(modes, ins, outs):
+        agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging, stream=s, pipelined=pipelined)
+    s.synchronize()
+    for k, ((hY, hdX, hdw), (Y, dX, dw)) in enumerate(zip(outs, refs)):
+        assert torch.equal(hY.view(torch.int16), Y.view(torch.int16)), k
+        assert torch.equal(hdX.view(torch.int16), dX.view(torch.int16)), k
+        assert torch.equal(hdw, dw), k
+
+
 def test_errors_are_reported_not_launched(agb):
     N, src, dst = skewed_edges(N=300, E=2000)
     wl, g = graph(agb, N, src, dst, 8)
