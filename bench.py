@@ -150,6 +150,11 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
+def dram_frac(dram_bytes, ms, peak_gbs):
+    """Measured DRAM bytes per call over the call's time, as a fraction of the peak."""
+    return dram_bytes / (ms / 1e3) / 1e9 / peak_gbs
+
+
 def traffic_key(args):
     return args.workload if args.rmat_scale is None else f"{args.workload}@scale{args.rmat_scale}"
 
@@ -477,6 +482,11 @@ def our_arm(args):
         gbs = algo[op] / (avg[op] / 1e3) / 1e9
         kernels[op] = {"ms": avg[op], "EH_per_s": wl.E * wl.H / (avg[op] / 1e3),
                        "algorithmic_bytes": algo[op], "GB_per_s": gbs, "frac_of_peak": gbs / hbm}
+        dram = ncu_traffic(traffic_key(args), op)
+        if dram:  # measured DRAM bytes of the call (ncu) over its live time: the DRAM fraction
+            kernels[op]["dram_bytes"] = dram
+            kernels[op]["dram_frac_of_peak"] = dram_frac(dram, avg[op], hbm)
+    traffic = ncu_traffic(traffic_key(args), dominant)
     launches_per_step = launches_per_step_of(st, wl)
     line = {
         "metric": METRIC,
@@ -491,7 +501,8 @@ def our_arm(args):
                      "peak": hbm, "unit": "GB/s",
                      "frac": algo[dominant] / (avg[dominant] / 1e3) / 1e9 / hbm,
                      "peak_source": f"{peak_kind} hbm_gbs",
-                     "traffic": ncu_traffic(traffic_key(args), dominant)},
+                     "traffic": traffic,
+                     "dram_frac": dram_frac(traffic, avg[dominant], hbm) if traffic else None},
         "kernels": kernels,
         "lowering_ms": lower_ms[1], "lowering_first_call_ms": lower_ms[0],
         "schedule": {k: st[k] for k in ("tile_edges", "tiles", "spanning_rows_f", "long_spanning_rows_f",

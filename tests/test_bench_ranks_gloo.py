@@ -109,3 +109,10 @@ def test_traffic_record_keys_on_code_not_comments():
     assert bench.code_only(src) == 'int a = 1;\n  const char *s = "// kept /* too */";\n  char c = \'"\';'
     assert bench.code_only("x = 1;\n// only a comment\n") == bench.code_only("x = 1;\n")
     assert bench.code_only("x = 1;") != bench.code_only("x = 2;")
+
+
+def test_dram_fraction():
+    sys.path.insert(0, ROOT)
+    import bench
+    # 11.42 GB in 3.16 ms against 6551.4 GB/s: about 55 %
+    assert abs(bench.dram_frac(11.42e9, 3.16, 6551.4) - 0.5516) < 1e-3
