@@ -324,6 +324,7 @@ def workload_config(wl, args):
             "l2": "inputs larger than L2 (X and dY exceed 126 MB), no flush" if wl.N * wl.H * (
                 2 if wl.feature_dtype == torch.bfloat16 else 4) > (126 << 20) else
                   "inputs smaller than L2: warm-L2 numbers",
+            "l2_persistence": "not set (no access policy window, default L2 set-aside)",
             "step": "ag_spmm_fwd + ag_backward (dX and dw fused) on a lowered graph; value = E*H per step / step time"}
 
 
