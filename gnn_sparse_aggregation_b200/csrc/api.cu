@@ -172,6 +172,6 @@ const char *ag_status_string(int status) {
     }
 }
 
-int ag_abi_version(void) { return 100; }
+int ag_abi_version(void) { return 101; }  // 1.01: ag_step_host_pipelined added
 
 }  // extern "C"
