@@ -348,6 +348,10 @@ AG_API int ag_step_host(const ag_graph *g, const float *w_host, const void *X_ho
  * an ag_step_host call on the same buffer keeps the order for the next
  * pipelined call.  The host input buffers are read until `stream` has been
  * synchronized after the call.
+ *
+ * Errors: those of ag_step_host (null buffers, staging too small or not
+ * 256-byte aligned, staging not on the graph's device, CUDA failures);
+ * AG_ERR_CUDA also when the ordering event cannot be created.
  */
 AG_API int ag_step_host_pipelined(const ag_graph *g, const float *w_host, const void *X_host,
                  const void *dY_host, void *Y_host, void *dX_host, float *dw_host,
