@@ -23,7 +23,11 @@
 //   5. the weight windows: every edge's slot in an order grouped by windows
 //      of 2^20 consecutive CSR positions (COO order inside a window), the
 //      slot read at every CSR position, and the per-chunk staging table that
-//      lets the per-call regrouping write whole runs of slots.
+//      lets the per-call regrouping write whole runs of slots.  An edge's
+//      window comes from its row's pointers (and, for the few rows that cross
+//      a window boundary, one order lookup); its slot from one ranking pass.
+// The radix scatter stages each tile in digit order in shared memory and
+// writes whole runs, so its global writes are coalesced.
 #include <climits>
 #include <cstdio>
 
@@ -37,6 +41,7 @@ constexpr int kRadixItems = 16;  // keys per thread
 constexpr int kRadixTile = kRadixThreads * kRadixItems;
 constexpr int kRadixWarps = kRadixThreads / 32;
 constexpr int kRadix = 256;
+static_assert(kRadixThreads == kRadix, "one thread per digit in the tile's digit scan");
 
 constexpr int kScanThreads = 256;
 constexpr int kScanItems = 8;
@@ -75,20 +80,52 @@ k_radix_hist(const int32_t *__restrict__ keys, int64_t n, int shift, int nblk,
         hist[int64_t(d) * nblk + blockIdx.x] = cnt[d];
 }
 
+// Exclusive scan of v over the kRadixThreads threads of the block (one value
+// each); returns this thread's prefix.  `wtot` holds kRadixWarps ints.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *wtot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wtot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+#pragma unroll
+    for (int w = 0; w < kRadixWarps; ++w) before += w < warp ? wtot[w] : 0;
+    __syncthreads();
+    return before + incl - v;
+}
+
 // Stable scatter of one digit pass.  Warp w of the tile owns the contiguous
-// items [w * 32 * kRadixItems, (w + 1) * 32 * kRadixItems) and walks them in
-// order, 32 at a time; offs holds the exclusive scan of hist.
+// items [w * 32 * kRadixItems, (w + 1) * 32 * kRadixItems) and ranks them in
+// order, 32 at a time (__match_any_sync inside a warp, warp order across the
+// tile), which gives every item its place in the tile's digit-sorted order;
+// offs holds the exclusive scan of hist (digit-major).
+//   MOVE: the tile is put in digit order in shared memory and then written
+//         out in that order, so that consecutive threads write consecutive
+//         addresses of one digit's run (keys_out, vals_out).
+//   otherwise: only the destination of every item is written, in item order:
+//         pos_out[i] = where item i goes (the rank of i in the stable order).
+template <bool MOVE>
 __global__ void __launch_bounds__(kRadixThreads)
 k_radix_scatter(const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in,
                 int64_t n, int shift, int nblk, const int32_t *__restrict__ offs,
                 int32_t *__restrict__ keys_out, int32_t *__restrict__ vals_out) {
     __shared__ int whist[kRadixWarps][kRadix];
+    __shared__ int dstart[kRadix];      // first place of each digit in the tile's sorted order
+    __shared__ int dbase[kRadix];       // global position of that place
+    __shared__ int wtot[kRadixWarps];
+    __shared__ int skey[MOVE ? kRadixTile : 1], sval[MOVE ? kRadixTile : 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < kRadixWarps * kRadix; i += kRadixThreads)
         (&whist[0][0])[i] = 0;
     __syncthreads();
 
-    const int64_t base = int64_t(blockIdx.x) * kRadixTile + int64_t(warp) * 32 * kRadixItems;
+    const int64_t tile0 = int64_t(blockIdx.x) * kRadixTile;
+    const int64_t base = tile0 + int64_t(warp) * 32 * kRadixItems;
     const unsigned lt = lanemask_lt();
     int key[kRadixItems], val[kRadixItems], rank[kRadixItems];
 #pragma unroll
@@ -110,25 +147,50 @@ k_radix_scatter(const int32_t *__restrict__ keys_in, const int32_t *__restrict__
         }
     }
     __syncthreads();
-    // exclusive prefix over warps, per digit: warp order = item order
-    for (int d = threadIdx.x; d < kRadix; d += kRadixThreads) {
-        int run = 0;
+    // exclusive prefix over warps, per digit (warp order = item order), and
+    // the tile's count of every digit
+    int count = 0;
+    {
+        const int d = threadIdx.x;  // kRadixThreads == kRadix
 #pragma unroll
         for (int w = 0; w < kRadixWarps; ++w) {
-            int t = whist[w][d];
-            whist[w][d] = run;
-            run += t;
+            const int t = whist[w][d];
+            whist[w][d] = count;
+            count += t;
         }
     }
+    const int start = block_exclusive_scan(count, wtot);
+    dstart[threadIdx.x] = start;
+    dbase[threadIdx.x] = offs[int64_t(threadIdx.x) * nblk + blockIdx.x];
     __syncthreads();
+    if constexpr (MOVE) {
 #pragma unroll
-    for (int k = 0; k < kRadixItems; ++k) {
-        const int64_t i = base + k * 32 + lane;
-        if (i < n) {
-            const int d = (uint32_t(key[k]) >> shift) & (kRadix - 1);
-            const int64_t pos = int64_t(offs[int64_t(d) * nblk + blockIdx.x]) + whist[warp][d] + rank[k];
-            keys_out[pos] = key[k];
-            vals_out[pos] = val[k];
+        for (int k = 0; k < kRadixItems; ++k) {
+            const int64_t i = base + k * 32 + lane;
+            if (i < n) {
+                const int d = (uint32_t(key[k]) >> shift) & (kRadix - 1);
+                const int local = dstart[d] + whist[warp][d] + rank[k];
+                skey[local] = key[k];
+                sval[local] = val[k];
+            }
+        }
+        __syncthreads();
+        const int m = int(n - tile0 < kRadixTile ? n - tile0 : kRadixTile);
+        for (int i = threadIdx.x; i < m; i += kRadixThreads) {
+            const int kk = skey[i];
+            const int d = (uint32_t(kk) >> shift) & (kRadix - 1);
+            const int64_t pos = int64_t(dbase[d]) + (i - dstart[d]);
+            keys_out[pos] = kk;
+            vals_out[pos] = sval[i];
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < kRadixItems; ++k) {
+            const int64_t i = base + k * 32 + lane;
+            if (i < n) {
+                const int d = (uint32_t(key[k]) >> shift) & (kRadix - 1);
+                vals_out[i] = dbase[d] + whist[warp][d] + rank[k];
+            }
         }
     }
 }
@@ -225,11 +287,21 @@ __global__ void k_rowptr_search(const int32_t *__restrict__ keys, int64_t E, int
     }
 }
 
+// out[i] = from[idx[i]]; four independent gathers in flight per thread
 __global__ void k_gather(const int32_t *__restrict__ idx, const int32_t *__restrict__ from,
                          int64_t n, int32_t *__restrict__ out) {
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
-         i += int64_t(gridDim.x) * blockDim.x)
-        out[i] = from[idx[i]];
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    for (; i + 3 * stride < n; i += 4 * stride) {
+        const int j0 = __ldcs(idx + i), j1 = __ldcs(idx + i + stride);
+        const int j2 = __ldcs(idx + i + 2 * stride), j3 = __ldcs(idx + i + 3 * stride);
+        const int v0 = from[j0], v1 = from[j1], v2 = from[j2], v3 = from[j3];
+        __stcs(out + i, v0);
+        __stcs(out + i + stride, v1);
+        __stcs(out + i + 2 * stride, v2);
+        __stcs(out + i + 3 * stride, v3);
+    }
+    for (; i < n; i += stride) out[i] = from[idx[i]];
 }
 
 __global__ void k_max_degree(const int32_t *__restrict__ rowptr, int64_t N, int *maxdeg) {
@@ -299,6 +371,27 @@ __global__ void k_span_scatter(const int32_t *__restrict__ nz_rows, const int32_
         const int4 v = make_int4(nz_rows[i], int(ta), int(tb), 0);
         if (tb - ta > kLongSpanTiles) spans[lpos[i]] = v;
         else spans[n_long + spos[i]] = v;
+    }
+}
+
+// out[e] = the weight window (position >> shift) of COO ordinal e, found from
+// its row key[e]: the row's positions [rowptr[k], rowptr[k + 1]) lie in one
+// window unless the row crosses window boundaries, and inside a row the
+// ordinals ascend with the position, so e lies at or past boundary B exactly
+// when order[B] <= e.  Reads are sequential except the L2-resident row
+// pointers.
+__global__ void k_window_of(const int32_t *__restrict__ key, const int32_t *__restrict__ rowptr,
+                            const int32_t *__restrict__ order, int64_t n, int shift, int32_t *__restrict__ out) {
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n;
+         e += int64_t(gridDim.x) * blockDim.x) {
+        const int k = __ldcs(key + e);
+        const int64_t a = rowptr[k], b = rowptr[k + 1];
+        int w = int(a >> shift);
+        for (int64_t B = (int64_t(w) + 1) << shift; B < b; B += int64_t(1) << shift) {
+            if (order[B] <= e) ++w;
+            else break;
+        }
+        __stcs(out + e, w);
     }
 }
 
@@ -414,7 +507,7 @@ const int32_t *radix_sort(const int32_t *keys_in, const int32_t *vals_in, int64_
         int32_t *vout = (p == passes - 1) ? vals_out : bufv[p & 1];
         k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(kin, n, 8 * p, nblk, t.hist);
         exclusive_scan(t.hist, t.hist, int64_t(kRadix) * nblk, t.scan, s);
-        k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(kin, vin, n, 8 * p, nblk, t.hist, kout, vout);
+        k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(kin, vin, n, 8 * p, nblk, t.hist, kout, vout);
         kin = kout;
         vin = vout;
     }
@@ -509,14 +602,27 @@ extern "C" int ag_graph_lower(const int32_t *src, const int32_t *dst, int64_t N,
         k_rowptr_search<<<grid_for(N + 1, 256), 256, 0, s>>>(sorted, E, N, D.rowptr);
         if (E > 0) k_gather<<<grid_for(E, 256), 256, 0, s>>>(D.order, other, E, D.col);
 
-        // window-bucketed weight layout (see kWindowShift): sort the COO
-        // ordinals stably by the window of their CSR position
+        // window-bucketed weight layout (see kWindowShift): the slot of an
+        // ordinal is its place in the COO ordinals sorted stably by the window
+        // of their CSR position
         if (E > 0) {
             int32_t *A = I(L.bucket_a[d]), *B = I(L.bucket_b[d]);
-            k_window_keys<<<grid_for(E, 256), 256, 0, s>>>(D.order, E, kWindowShift, A);
-            radix_sort(A, nullptr, E, bit_length((E - 1) >> kWindowShift), B, t, s);  // B[slot] = ordinal
-            k_invert<<<grid_for(E, 256), 256, 0, s>>>(B, E, A);                        // A[ordinal] = slot
-            k_gather<<<grid_for(E, 256), 256, 0, s>>>(D.order, A, E, B);              // B[pos] = slot
+            const int wbits = bit_length((E - 1) >> kWindowShift);
+            if (wbits <= 8) {
+                // windows from the row pointers (the sorted keys are dead), then
+                // one ranking pass: A[ordinal] = its place in the stable order
+                int32_t *win = t.keys_a;
+                k_window_of<<<grid_for(E, 256), 256, 0, s>>>(key, D.rowptr, D.order, E, kWindowShift, win);
+                const int nblk = int((E + kRadixTile - 1) / kRadixTile);
+                k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(win, E, 0, nblk, t.hist);
+                exclusive_scan(t.hist, t.hist, int64_t(kRadix) * nblk, t.scan, s);
+                k_radix_scatter<false><<<nblk, kRadixThreads, 0, s>>>(win, nullptr, E, 0, nblk, t.hist, nullptr, A);
+            } else {
+                k_window_keys<<<grid_for(E, 256), 256, 0, s>>>(D.order, E, kWindowShift, A);
+                radix_sort(A, nullptr, E, wbits, B, t, s);              // B[slot] = ordinal
+                k_invert<<<grid_for(E, 256), 256, 0, s>>>(B, E, A);     // A[ordinal] = slot
+            }
+            k_gather<<<grid_for(E, 256), 256, 0, s>>>(D.order, A, E, B);  // B[pos] = slot
             D.bucket_of_coo = A;
             D.bucket_of_pos = B;
             if (staged_regroup(E)) {
