@@ -376,9 +376,11 @@ AG_API int ag_step_host_pipelined(const ag_graph *g, const float *w_host, const 
  *     launched.
  *   - The call allocates nothing (no cudaMalloc, cudaFree or allocating
  *     library routine).  Its first call on a device looks up the array's
- *     device address there (cudaGetSymbolAddress); make that first call
- *     before any stream capture.  Call it with the graph's device current
- *     (AG_ERR_DEVICE otherwise).
+ *     device address there (cudaGetSymbolAddress) and keeps it for the life
+ *     of the process; make that first call before any stream capture, and do
+ *     not reset the device (cudaDeviceReset) while the library is loaded,
+ *     since the kept address would then be stale.  Call it with the graph's
+ *     device current (AG_ERR_DEVICE otherwise).
  *   - All calls share the one array: calls whose work overlaps on the GPU
  *     (different streams, different host threads) race and must be ordered
  *     by the caller.  The array keeps the previous call's contents; no part
