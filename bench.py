@@ -305,7 +305,7 @@ def reference_arm(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": workload_config(wl, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"first {S} of {wl.E} COO edges (endpoints relabelled), "
                                    f"fwd+dX+dw per step, H={wl.H}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -446,7 +446,7 @@ def our_arm(args):
 
     # end to end from host buffers, copies inside the timed region
     e2e = None
-    Ke = args.e2e_steps if args.e2e_steps is not None else min(K, 5)
+    Ke = args.e2e_steps if args.e2e_steps is not None else min(K, 20)
     if Ke > 0:
         hw, hX, hdY = (t.cpu().pin_memory() for t in (wl.w, wl.X, wl.dY))
         hY, hdX = torch.empty_like(hX).pin_memory(), torch.empty_like(hX).pin_memory()
@@ -520,7 +520,8 @@ def our_arm(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         S, sample, run = oracle_sample(wl, args.cpu_seconds)
         secs = run(sample)
-        line["cpu_baseline"] = {"value": S * wl.H / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
+        line["cpu_baseline"] = {"value": S * wl.H / secs, "unit": UNIT, "cores": 1, "host_cores": os.cpu_count(),
+                                "kind": "oracle",
                                 "sample": f"first {S} of {wl.E} COO edges (endpoints relabelled), "
                                           f"one fwd+dX+dw pass, H={wl.H}, {secs:.1f} s"}
     if rank == 0:

@@ -154,8 +154,19 @@ def test_unaligned_feature_pointers_take_the_narrow_path(agb, dtype):
     Y = g.fwd(wl.w, Xu)
     ref = g.fwd(wl.w, wl.X)
     torch.cuda.synchronize()
-    # different vector widths keep the same per-element order of operations
-    assert torch.equal(Y.float(), ref.float())
+    # The aligned input takes the paired walk, which sums the even and the odd
+    # positions of a row in the two halves of a warp and adds the two sums at
+    # the row end; the unaligned one takes a narrower walk that sums in
+    # position order.  Any summation order is acceptable within the tolerance
+    # (fp32 accumulation against the fp64 oracle), so both are checked there,
+    # and each must reproduce itself bit for bit.
+    import oracle
+    want, bound = oracle.fwd(host(wl.src), host(wl.dst), N, host(wl.w), host(wl.X), with_bound=True)
+    assert_within(Y, want, bound, TOL[dtype], "narrow path")
+    assert_within(ref, want, bound, TOL[dtype], "wide path")
+    Y2 = g.fwd(wl.w, Xu)
+    torch.cuda.synchronize()
+    assert torch.equal(Y2.float(), Y.float())
 
 
 def _rows_per_tile_graph(kind, rng):
@@ -360,6 +371,37 @@ def test_pipelined_steps_keep_each_steps_results(agb, modes):
     for k, ((hY, hdX, hdw), (Y, dX, dw)) in enumerate(zip(outs, refs)):
         assert torch.equal(hY.view(torch.int16), Y.view(torch.int16)), k
         assert torch.equal(hdX.view(torch.int16), dX.view(torch.int16)), k
+        assert torch.equal(hdw, dw), k
+
+
+def test_pipelined_steps_with_a_new_layout_on_the_same_buffer(agb):
+    """Pipelined steps of different widths (and dtypes) back to back on one
+    staging buffer: a step whose layout differs from the previous step's must
+    not start its copies in before the previous step's copies out are done
+    (its input part overlaps the previous step's output part), so every step
+    still returns exactly what ag_step_host returns for it alone."""
+    src, dst = workloads.rmat_edges(16, 16, seed=7)
+    N = 1 << 16
+    shapes = ((128, torch.bfloat16), (32, torch.float32), (64, torch.bfloat16), (128, torch.bfloat16))
+    g = agb.ag_graph_lower(torch.from_numpy(src.numpy()).to(DEV), torch.from_numpy(dst.numpy()).to(DEV), N)
+    big = max(agb.ag_step_staging_bytes(g, H, dt) for H, dt in shapes)
+    staging = torch.empty(big, dtype=torch.uint8, device=DEV)
+    ins, outs, refs = [], [], []
+    for k, (H, dt) in enumerate(shapes):
+        wl = workloads.custom(N, src.numpy(), dst.numpy(), H, seed=20 + k, feature_dtype=dt, device=DEV)
+        refs.append(tuple(t.cpu() for t in (g.fwd(wl.w, wl.X), *g.backward(wl.w, wl.X, wl.dY))))
+        ins.append(tuple(t.cpu().pin_memory() for t in (wl.w, wl.X, wl.dY)))
+        outs.append((torch.empty_like(ins[-1][1]).pin_memory(), torch.empty_like(ins[-1][1]).pin_memory(),
+                     torch.empty_like(ins[-1][0]).pin_memory()))
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    for (hw, hX, hdY), (hY, hdX, hdw) in zip(ins, outs):
+        agb.ag_step_host(g, hw, hX, hdY, hY, hdX, hdw, staging, stream=s, pipelined=True)
+    s.synchronize()
+    for k, ((hY, hdX, hdw), (Y, dX, dw)) in enumerate(zip(outs, refs)):
+        bits = (lambda t: t.view(torch.int16)) if Y.dtype == torch.bfloat16 else (lambda t: t.view(torch.int32))
+        assert torch.equal(bits(hY), bits(Y)), k
+        assert torch.equal(bits(hdX), bits(dX)), k
         assert torch.equal(hdw, dw), k
 
 
