@@ -57,6 +57,9 @@ def parse_args():
     p.add_argument("--no-rows", action="store_true",
                    help="skip the timings of mean, GCN weights and attention reported beside the step")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time per sample")
+    p.add_argument("--profile-once", action="store_true",
+                   help="lower the graph once and call every entry point once, without timing "
+                        "(a short launch sequence for profilers)")
     return p.parse_args()
 
 
@@ -328,6 +331,42 @@ def workload_config(wl, args):
             "step": "ag_spmm_fwd + ag_backward (dX and dw fused) on a lowered graph; value = E*H per step / step time"}
 
 
+def profile_once(args):
+    """One lowering, then each entry point once (step calls, the separate
+    gradients, mean, GCN weights weighted and unweighted, attention forward
+    and backward), in that order, with a synchronize at the end."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    from __graft_entry__ import build_library
+    build_library()
+    import gnn_sparse_aggregation_b200 as agb
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = workloads.make(args.workload, seed=args.seed, device=dev, rmat_scale=args.rmat_scale)
+    g = agb.ag_graph_lower(wl.src, wl.dst, wl.N)
+    Y, dX = torch.empty_like(wl.X), torch.empty_like(wl.dY)
+    dw, wn = torch.empty_like(wl.w), torch.empty_like(wl.w)
+    mk = lambda s: workloads.features(wl.N, wl.H, wl.feature_dtype, 11000 + s, dev)
+    Q, Kf, V = mk(1), mk(2), mk(3)
+    Ya, dQ, dK, dV = (torch.empty_like(wl.X) for _ in range(4))
+    alpha = torch.empty(wl.E, dtype=torch.float32, device=dev)
+    scale = 1.0 / wl.H ** 0.5
+    agb.ag_spmm_fwd(g, wl.w, wl.X, Y)
+    agb.ag_backward(g, wl.w, wl.X, wl.dY, dX, dw)
+    agb.ag_spmm_dx(g, wl.w, wl.dY, dX)
+    agb.ag_sddmm_dw(g, wl.X, wl.dY, dw)
+    agb.ag_mean_fwd(g, wl.w, wl.X, Y)
+    agb.ag_mean_backward(g, wl.w, wl.X, wl.dY, dX, dw)
+    agb.ag_gcn_norm(g, wl.w, wn)
+    agb.ag_gcn_norm(g, None, wn)
+    agb.ag_attn_fwd(g, Q, Kf, V, scale, Ya, alpha)
+    agb.ag_attn_backward(g, Q, Kf, V, scale, alpha, wl.dY, dQ, dK, dV)
+    torch.cuda.synchronize()
+    print(f"profile-once done: {wl.name} N={wl.N} E={wl.E} H={wl.H}", flush=True)
+    g.close()
+    return 0
+
+
 def our_arm(args):
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -536,6 +575,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return reference_arm(args)
+    if args.profile_once:
+        return profile_once(args)
     return our_arm(args)
 
 

@@ -53,6 +53,9 @@ namespace {
 #ifndef AG_CHUNK
 #define AG_CHUNK 8        // positions per unrolled chunk of a gradient-walk batch (the rest is rolled)
 #endif
+#ifndef AG_WALK
+#define AG_WALK 1         // 1: rows of 1024 bytes take the warp walk (k_walk)
+#endif
 #ifndef AG_MAX_LANES
 #define AG_MAX_LANES 16   // lanes that share one row (fewer lanes: more 16-byte vectors per lane)
 #endif
@@ -679,6 +682,347 @@ k_tiles_ring(const Params P) {
     cp_async_wait<0>();
 }
 
+// ---------------------------------------------------------------------------- warp walk: one warp per tile
+
+// The walk for rows of 1024 bytes (fp32 H = 256, bf16 H = 512), which the
+// ring walk would hold as four 16-byte vectors per lane.  One warp walks one
+// tile, one CSR position at a time, and every lane owns 32 bytes of each row
+// (two 16-byte segments).  Gathered rows travel global -> shared memory with
+// cp.async into a per-warp ring of D = 4 rows (4 KB per warp), so that a warp
+// keeps D rows in flight without holding them in registers; each lane copies,
+// and later reads, only its own bytes of every row, so no barrier is needed
+// between copy and read.  (Rows are not moved by the tensor memory
+// accelerator: per-row cp.async.bulk and tile::gather4 copies gathered random
+// 256-byte rows at 1-4.4 TB/s on B200, plain loads at about 15 TB/s.)
+// All 32 lanes work on the same position, so the row-end test, the weight
+// and the column index are warp-uniform: a batch of 32 positions that lies
+// inside one row runs without any test, in unrolled chunks of 8 positions;
+// the others run one position at a time with the row-end test.
+//   kSpmm : out[row] = sum w[slot(p)] * F[col[p]] over the row's positions
+//   kSddmm: dw[slot(p)] = dot(R[row], F[col[p]]); the per-lane partial dots of
+//           a chunk of 8 positions are reduced with one reduce-scatter (one
+//           butterfly per position in the batches with row ends), after which
+//           lane p % 32 writes the weight gradient of position p
+//   kBoth : both on one walk of the transpose CSR
+// Owner rows (kSddmm) are loaded kOwnAhead rows ahead of their first use;
+// the next 64 rows' ids and ends are held in two 32-row windows, one lane per
+// row, the second loaded while the first is used.  Rows cut by a tile
+// boundary leave partial rows exactly as in k_tiles (slot 2t: continued from
+// the previous tile, 2t + 1: continued in the next), summed by k_fixup.
+
+// This lane's LB bytes of a row: NSEG segments of SEGB bytes, segment q of
+// lane l at byte q * 32 * SEGB + l * SEGB, so that a warp-wide access of one
+// segment touches 32 * SEGB consecutive bytes.
+template <int LB> struct Slice {
+    static_assert(LB % 16 == 0, "16-byte segments");
+    static constexpr int SEGB = 16;
+    static constexpr int NSEG = LB / SEGB;
+    static constexpr int NW = LB / 4;
+    uint32_t w[NW];
+};
+
+template <int LB>
+__device__ __forceinline__ void load_slice(const char *p, Slice<LB> &s) {
+#pragma unroll
+    for (int q = 0; q < Slice<LB>::NSEG; ++q) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p + q * 32 * 16));
+        s.w[4 * q] = v.x;
+        s.w[4 * q + 1] = v.y;
+        s.w[4 * q + 2] = v.z;
+        s.w[4 * q + 3] = v.w;
+    }
+}
+// the same from this lane's bytes of a ring slot
+template <int LB>
+__device__ __forceinline__ void lds_slice(const char *p, Slice<LB> &s) {
+#pragma unroll
+    for (int q = 0; q < Slice<LB>::NSEG; ++q) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p + q * 32 * 16);
+        s.w[4 * q] = v.x;
+        s.w[4 * q + 1] = v.y;
+        s.w[4 * q + 2] = v.z;
+        s.w[4 * q + 3] = v.w;
+    }
+}
+// copy this lane's bytes of a row (src: row start + lane offset) to a ring slot
+template <int LB>
+__device__ __forceinline__ void cp_async_slice(uint32_t dst, const char *src) {
+#pragma unroll
+    for (int q = 0; q < Slice<LB>::NSEG; ++q) cp_async16(dst + q * 32 * 16, src + q * 32 * 16);
+}
+
+// fp32 values of a slice, in feature order within each segment
+template <typename T, int LB>
+__device__ __forceinline__ void unpack_slice(const Slice<LB> &s, float (&v)[LB / sizeof(T)]) {
+    if constexpr (sizeof(T) == 4) {
+#pragma unroll
+        for (int k = 0; k < Slice<LB>::NW; ++k) v[k] = __uint_as_float(s.w[k]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < Slice<LB>::NW; ++k) {
+            v[2 * k] = bf16_lo(s.w[k]);
+            v[2 * k + 1] = bf16_hi(s.w[k]);
+        }
+    }
+}
+
+// Output row slice in the feature dtype (streaming stores: written once).
+template <typename T, int LB>
+__device__ __forceinline__ void store_slice(char *p, const float (&v)[LB / sizeof(T)]) {
+    uint32_t w[Slice<LB>::NW];
+#pragma unroll
+    for (int k = 0; k < Slice<LB>::NW; ++k)
+        w[k] = sizeof(T) == 4 ? __float_as_uint(v[k]) : pack_bf16(v[2 * k], v[2 * k + 1]);
+#pragma unroll
+    for (int q = 0; q < Slice<LB>::NSEG; ++q)
+        __stcs(reinterpret_cast<uint4 *>(p + q * 32 * 16), make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
+}
+
+// The same slice as fp32 partial sums, at the same feature indices of a
+// partial row [H] (what k_fixup adds up).
+template <typename T, int LB>
+__device__ __forceinline__ void store_slice_partial(float *row, int lane, const float (&v)[LB / sizeof(T)]) {
+    constexpr int SEGB = Slice<LB>::SEGB, VPS = SEGB / int(sizeof(T));
+#pragma unroll
+    for (int q = 0; q < Slice<LB>::NSEG; ++q) {
+        float *d = row + (q * 32 * SEGB + lane * SEGB) / int(sizeof(T));
+#pragma unroll
+        for (int i = 0; i < VPS; i += 4)
+            *reinterpret_cast<float4 *>(d + i) =
+                make_float4(v[q * VPS + i], v[q * VPS + i + 1], v[q * VPS + i + 2], v[q * VPS + i + 3]);
+    }
+}
+
+constexpr int kZeroRowsPerWarp = 8;  // empty rows zeroed by each of the trailing warps
+constexpr int kOwnAhead = 2;         // owner rows loaded ahead of their first use (gradient walks)
+constexpr int kWalkRingBytes = 4096;  // ring bytes per warp: D = kWalkRingBytes / row bytes rows in flight
+
+// ids and ends of the non-empty rows base .. base + 31 (one per lane);
+// past the last row: row 0 (a valid address) and an end no position reaches
+__device__ __forceinline__ void load_rows(const Params &P, int64_t base, int lane, int &row, int &end) {
+    row = 0;
+    end = INT_MAX;
+    if (base + lane < P.n_nz) {
+        row = __ldg(P.nz_rows + base + lane);
+        end = __ldg(P.nz_rowptr + base + lane + 1);
+    }
+}
+
+// resident CTAs per SM the walk is compiled for (a register budget)
+constexpr int walk_min_blocks(int MODE) { return (MODE & kSddmm) ? 2 : 4; }
+
+template <typename T, int LB, int MODE>
+__global__ void __launch_bounds__(kThreads, walk_min_blocks(MODE)) k_walk(const Params P) {
+    using S = Slice<LB>;
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int VPL = LB / int(sizeof(T));
+    constexpr int RB = 32 * LB;
+    constexpr int D = kWalkRingBytes / RB;  // rows in flight per warp
+    constexpr int CH = 8;                   // positions per unrolled chunk (and per reduction of partial dots)
+    static_assert(32 % D == 0 && (D >= CH ? D % CH == 0 : CH % D == 0), "chunk shapes");
+    constexpr bool SPMM = (MODE & kSpmm) != 0, SDDMM = (MODE & kSddmm) != 0;
+    constexpr bool ROW_SCALE = (MODE & kRowScale) != 0, EDGE_SCALE = (MODE & kEdgeScale) != 0;
+    extern __shared__ uint4 walk_ring[];  // (kThreads / 32) * kWalkRingBytes bytes
+    char *ring = reinterpret_cast<char *>(walk_ring);
+
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int lane_off = lane * S::SEGB;
+    if (warp >= P.n_tiles) {  // trailing warps: rows without edges get zeros
+        const int64_t z0 = (warp - P.n_tiles) * kZeroRowsPerWarp;
+        float zero[VPL];
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) zero[v] = 0.f;
+        for (int k = 0; k < kZeroRowsPerWarp && z0 + k < P.n_zero; ++k)
+            store_slice<T, LB>(static_cast<char *>(P.out) + int64_t(P.zero_rows[z0 + k]) * RB + lane_off, zero);
+        return;
+    }
+    // this lane's bytes of ring slot s: my + s * RB (shared address my_s + s * RB)
+    const char *my = ring + (threadIdx.x >> 5) * kWalkRingBytes + lane_off;
+    const uint32_t my_s = smem_addr(my);
+
+    const int p0 = int(warp * P.T);
+    const int pend = int(min(int64_t(p0) + P.T, P.E));
+    const char *__restrict__ F = static_cast<const char *>(P.F) + lane_off;
+    const char *__restrict__ R = static_cast<const char *>(P.R) + lane_off;
+    char *__restrict__ out = static_cast<char *>(P.out) + lane_off;
+    float *slot_head = P.partial + (2 * warp) * P.H;
+    float *slot_tail = P.partial + (2 * warp + 1) * P.H;
+
+    // the open row, and the next 64 rows in two windows (a: next 32, b: the 32 after)
+    int64_t ci = P.tile_nz[warp];
+    int row = __ldg(P.nz_rows + ci);
+    int rend = __ldg(P.nz_rowptr + ci + 1);
+    bool before = __ldg(P.nz_rowptr + ci) < p0;
+    int64_t wbase = ci + 1;
+    int wa_row, wa_end, wb_row, wb_end;
+    load_rows(P, wbase, lane, wa_row, wa_end);
+    load_rows(P, wbase + 32, lane, wb_row, wb_end);
+    int wk = 0;  // the next row is window a, lane wk
+
+    // column index and weight slot of batch b (cur), b + 1 (nxt); weights of b
+    int c_cur = 0, s_cur = 0, c_nxt = 0, s_nxt = 0;
+    if (p0 + lane < pend) {
+        c_cur = __ldcs(P.col + p0 + lane);
+        s_cur = __ldcs(P.order + p0 + lane);
+    }
+    if (p0 + 32 + lane < pend) {
+        c_nxt = __ldcs(P.col + p0 + 32 + lane);
+        s_nxt = __ldcs(P.order + p0 + 32 + lane);
+    }
+    float w_cur = 0.f;
+    if (SPMM && p0 + lane < pend) {
+        w_cur = load_w(P.w + s_cur);
+        if constexpr (EDGE_SCALE) w_cur *= __ldg(P.inv_cnt + c_cur);
+    }
+
+    // rows in flight: positions b0 + j .. b0 + j + D - 1, slot = position mod D,
+    // one cp.async group per position (empty past the tile's end)
+#pragma unroll
+    for (int u = 0; u < D; ++u) {
+        cp_async_slice<LB>(my_s + u * RB, F + int64_t(__shfl_sync(FULL, c_cur, u)) * RB);
+        cp_async_commit();
+    }
+
+    float acc[VPL], own[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc[v] = 0.f, own[v] = 0.f;
+    S oq[kOwnAhead];  // owner rows of window a, lanes wk .. wk + kOwnAhead - 1
+    if constexpr (SDDMM) {
+        S o;
+        load_slice<LB>(R + int64_t(row) * RB, o);
+        unpack_slice<T, LB>(o, own);
+#pragma unroll
+        for (int k = 0; k < kOwnAhead; ++k) load_slice<LB>(R + int64_t(__shfl_sync(FULL, wa_row, k)) * RB, oq[k]);
+    }
+
+    auto flush = [&](float *slot) {
+        if (slot) {
+            store_slice_partial<T, LB>(slot, lane, acc);
+        } else {
+            if constexpr (ROW_SCALE) {
+                const float r = __ldg(P.inv_cnt + row);
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) acc[v] *= r;
+            }
+            store_slice<T, LB>(out + int64_t(row) * RB, acc);
+        }
+    };
+    // the open row ended at the current position: write it, open the next
+    auto next_row = [&]() {
+        if constexpr (SPMM) {
+            flush(before ? slot_head : nullptr);
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
+        }
+        before = false;
+        if constexpr (SDDMM) {
+            unpack_slice<T, LB>(oq[0], own);
+#pragma unroll
+            for (int k = 0; k + 1 < kOwnAhead; ++k) oq[k] = oq[k + 1];
+            const int k = wk + kOwnAhead;
+            const int r = __shfl_sync(FULL, k < 32 ? wa_row : wb_row, k & 31);
+            load_slice<LB>(R + int64_t(r) * RB, oq[kOwnAhead - 1]);
+        }
+        row = __shfl_sync(FULL, wa_row, wk);
+        rend = __shfl_sync(FULL, wa_end, wk);
+        if (++wk == 32) {
+            wa_row = wb_row;
+            wa_end = wb_end;
+            wk = 0;
+            wbase += 32;
+            load_rows(P, wbase + 32, lane, wb_row, wb_end);
+        }
+    };
+
+    float dots[CH];
+#pragma unroll
+    for (int t = 0; t < CH; ++t) dots[t] = 0.f;
+    // Position b0 + j (held in ring slot `slot`): returns this lane's part of
+    // its dot product (SDDMM); CHECK: test the tile end and the row end.
+    auto position = [&](int b0, int j, int slot, bool check) -> float {
+        const bool valid = !check || b0 + j < pend;
+        cp_async_wait<D - 1>();  // the group of this position has landed
+        if (check && valid && b0 + j == rend) next_row();
+        S xs;
+        lds_slice<LB>(my + slot * RB, xs);
+        float xv[VPL];
+        unpack_slice<T, LB>(xs, xv);
+        if constexpr (SPMM) {
+            const float wj = __shfl_sync(FULL, w_cur, j & 31);
+            if (valid) {
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) acc[v] = fmaf(wj, xv[v], acc[v]);
+            }
+        }
+        float d = 0.f;
+        if constexpr (SDDMM) {
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) d = fmaf(own[v], xv[v], d);
+        }
+        // refill the slot with position b0 + j + D (the column of a position
+        // past the tile's end is 0: a valid row, never read)
+        const int jn = j + D;
+        const int src = __shfl_sync(FULL, jn < 32 ? c_cur : c_nxt, jn & 31);
+        cp_async_slice<LB>(my_s + slot * RB, F + int64_t(src) * RB);
+        cp_async_commit();
+        return valid ? d : 0.f;
+    };
+
+    for (int b0 = p0; b0 < pend; b0 += 32) {
+        // indices of batch b + 2 (prefetched, consumed next batch), weights of batch b + 1
+        int c_nn = 0, s_nn = 0;
+        if (b0 + 64 + lane < pend) {
+            c_nn = __ldcs(P.col + b0 + 64 + lane);
+            s_nn = __ldcs(P.order + b0 + 64 + lane);
+        }
+        float w_nxt = 0.f;
+        if (SPMM && b0 + 32 + lane < pend) {
+            w_nxt = load_w(P.w + s_nxt);
+            if constexpr (EDGE_SCALE) w_nxt *= __ldg(P.inv_cnt + c_nxt);
+        }
+        if (b0 + 32 <= pend && rend >= b0 + 32) {
+            // the whole batch lies in the open row: chunks of CH positions
+            // without tests; the CH partial dots of a chunk are reduced with
+            // one reduce-scatter, after which lane j of the chunk's lane block
+            // holds the dot of position b0 + lane and writes it
+#pragma unroll 1
+            for (int c = 0; c < 32; c += CH) {
+                const int sb = c % D;  // slots sb .. sb + CH - 1 (mod D) hold the chunk
+#pragma unroll
+                for (int t = 0; t < CH; ++t) dots[t] = position(b0, c + t, D >= CH ? sb + t : t % D, false);
+                if constexpr (SDDMM) {
+                    const float d = reduce_chunk<CH, 32>(dots, lane, FULL);
+                    if ((lane & ~(CH - 1)) == c) P.dw[s_cur] = EDGE_SCALE ? d * __ldg(P.inv_cnt + c_cur) : d;
+                }
+            }
+        } else {
+            // one position at a time with the row-end test; each dot is
+            // reduced over the warp on its own and written by lane j
+#pragma unroll 1
+            for (int j = 0; j < 32; ++j) {
+                float d = position(b0, j, j % D, true);
+                if constexpr (SDDMM) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
+                    if (lane == j && b0 + j < pend) P.dw[s_cur] = EDGE_SCALE ? d * __ldg(P.inv_cnt + c_cur) : d;
+                }
+            }
+        }
+        c_cur = c_nxt;
+        s_cur = s_nxt;
+        w_cur = w_nxt;
+        c_nxt = c_nn;
+        s_nxt = s_nn;
+    }
+    if constexpr (SPMM) {
+        if (before) flush(slot_head);
+        else if (rend > pend) flush(slot_tail);
+        else flush(nullptr);
+    }
+    cp_async_wait<0>();
+}
+
 template <int VEC, int NV>
 __device__ __forceinline__ void scale_rows(float (&acc)[NV][VEC], float r) {
 #pragma unroll
@@ -782,6 +1126,7 @@ k_fixup(const int4 *__restrict__ spans, int64_t n_long, int64_t n_span, const fl
 
 struct Shape {
     int vec, G, log2G, nv, col_tiles;
+    int lb;  // > 0: bytes per lane of the register walk (rows of 32 * lb bytes)
 };
 
 int log2i(int v) {
@@ -818,6 +1163,11 @@ Shape pick_shape(int64_t H, int dtype, const void *a, const void *b, const void 
     const int64_t per_lane = (HV + G - 1) / G;
     s.nv = per_lane <= 1 ? 1 : (per_lane <= 2 ? 2 : 4);
     s.col_tiles = int((HV + int64_t(G) * s.nv - 1) / (int64_t(G) * s.nv));
+    // the warp walk: rows of 1024 bytes (fp32 H = 256, bf16 H = 512), every
+    // pointer 16-byte aligned; narrower rows take the shared-memory ring walk
+    const int64_t row_bytes = H * elem;
+    s.lb = 0;
+    if (AG_WALK && row_bytes == 1024 && aligned(a, 16) && aligned(b, 16) && aligned(c, 16)) s.lb = 32;
     return s;
 }
 
@@ -884,8 +1234,36 @@ void dispatch_nv(const Params &P, const Shape &s, cudaStream_t st) {
     }
 }
 
+template <typename T, int LB, int MODE>
+void launch_walk(const Params &P, cudaStream_t st) {
+    const int64_t warps = P.n_tiles + (P.n_zero + kZeroRowsPerWarp - 1) / kZeroRowsPerWarp;
+    const unsigned grid = unsigned((warps + kThreads / 32 - 1) / (kThreads / 32));
+    const size_t smem = size_t(kThreads / 32) * kWalkRingBytes;
+    // the shared-memory limit is an attribute of the function in each device's
+    // context: set it once per device (a race only repeats the same call)
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = uint64_t(1) << (dev & 63);
+    if (!(configured.load(std::memory_order_relaxed) & bit)) {
+        cudaFuncSetAttribute(k_walk<T, LB, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        configured.fetch_or(bit, std::memory_order_relaxed);
+    }
+    if (grid > 0) k_walk<T, LB, MODE><<<grid, kThreads, smem, st>>>(P);
+}
+
+template <int MODE, typename T>
+void dispatch_walk(const Params &P, int lb, cudaStream_t st) {
+    launch_walk<T, 32, MODE>(P, st);  // pick_shape selects the warp walk for 1024-byte rows only
+}
+
 template <int MODE>
 void dispatch_main(const Params &P, const Shape &s, int dtype, cudaStream_t st) {
+    if (s.lb > 0) {
+        if (dtype == AG_F32) dispatch_walk<MODE, float>(P, s.lb, st);
+        else dispatch_walk<MODE, bf16_t>(P, s.lb, st);
+        return;
+    }
     if (dtype == AG_F32) {
         if (s.vec == 4) dispatch_nv<MODE, float, 4>(P, s, st);
         else dispatch_nv<MODE, float, 1>(P, s, st);
@@ -1136,7 +1514,7 @@ int check_scratch(const ag_graph *g, size_t need, const void *scratch, size_t sc
 // SpMM over direction d: out = A_w X (d = 0) or A_w^T dY (d = 1).
 // The shapes the shared-memory ring walks take (see launch_main).
 bool ring_shape(const Shape &s, int dtype, int64_t H) {
-    return s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8) &&
+    return s.lb > 0 || s.col_tiles == 1 && s.G >= 4 && s.nv <= 2 && (dtype == AG_F32 ? s.vec == 4 : s.vec == 8) &&
            int64_t(s.G) * s.nv * s.vec == H;
 }
 
@@ -1377,7 +1755,62 @@ int gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch, si
     return AG_OK;
 }
 
+// The SpMM walk over direction d with weights already in that direction's
+// window slots (no regrouping): out = A_w F (d = 0) or A_w^T F (d = 1).
+// scratch: an SpMM scratch of width H (its partial rows are used).
+int spmm_bucketed_impl(const ag_graph *g, int d, const float *w_b, const void *F, void *out, int64_t H, int dtype,
+                       void *scratch, cudaStream_t st) {
+    const ag::Direction &D = g->dir[d];
+    const ScratchLayout SL = scratch_layout(g, H);
+    const Shape s = pick_shape(H, dtype, F, out, nullptr);
+    Params P = base_params(g, D, H, s);
+    P.F = F;
+    P.out = out;
+    P.w = w_b;
+    P.order = D.bucket_of_pos;
+    P.partial = reinterpret_cast<float *>(static_cast<char *>(scratch) + SL.partial);
+    P.n_zero = g->N - D.n_nz;
+    if (P.n_tiles + P.n_zero > 0) dispatch_main<kSpmm>(P, s, dtype, st);
+    if (D.n_span > 0) dispatch_fixup(D, P.partial, out, H, s, dtype, st);
+    cudaError_t err = cudaGetLastError();
+    return err == cudaSuccess ? AG_OK : cuda_fail(err, "bucketed SpMM");
+}
+
+// The SDDMM walk over direction d: out_b[slot of position p] = dot(R[row of
+// p], F[col[p]]) in that direction's window slots (no regrouping).
+int sddmm_bucketed_impl(const ag_graph *g, int d, const void *R, const void *F, float *out_b, int64_t H, int dtype,
+                        cudaStream_t st) {
+    if (g->E == 0) return AG_OK;
+    const ag::Direction &D = g->dir[d];
+    const Shape s = pick_shape(H, dtype, R, F, nullptr);
+    Params P = base_params(g, D, H, s);
+    P.order = D.bucket_of_pos;
+    P.F = F;
+    P.R = R;
+    P.dw = out_b;
+    P.n_zero = 0;
+    dispatch_main<kSddmm>(P, s, dtype, st);
+    cudaError_t err = cudaGetLastError();
+    return err == cudaSuccess ? AG_OK : cuda_fail(err, "bucketed SDDMM");
+}
+
 }  // namespace
+
+int spmm_bucketed(const ag_graph *g, int d, const float *w_b, const void *F, void *out, int64_t H, int dtype,
+                  void *scratch, cudaStream_t st) {
+    return spmm_bucketed_impl(g, d, w_b, F, out, H, dtype, scratch, st);
+}
+int sddmm_bucketed(const ag_graph *g, int d, const void *R, const void *F, float *out_b, int64_t H, int dtype,
+                   cudaStream_t st) {
+    return sddmm_bucketed_impl(g, d, R, F, out_b, H, dtype, st);
+}
+void regroup_from_buckets(const ag_graph *g, int d, const float *in_b, float *out, cudaStream_t st) {
+    regroup(false, g->dir[d], in_b, g->E, out, st);
+}
+int backward_into(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw, int64_t H,
+                  int dtype, void *scratch, size_t scratch_bytes, cudaStream_t st) {
+    return backward(g, w, X, dY, dX, dw, H, dtype, scratch, scratch_bytes, st, "ag_attn_backward", false);
+}
 
 size_t spmm_scratch_edge_offset(const ag_graph *g, int64_t H, int which) {
     const ScratchLayout L = scratch_layout(g, H);
@@ -1494,48 +1927,67 @@ struct StepEvents {
 // Pipelined steps: per staging buffer, an event recorded after the last
 // read of its input part (w, X, dY) by a step's fused backward pass.  The
 // input copies of the next pipelined step on that buffer wait for this
-// event only, so they overlap the previous step's copies out.  A bounded
-// table: a buffer whose entry was reused, or that was never seen, gets the
-// full ordering after `stream` again.
+// event only, so they overlap the previous step's copies out.  That is safe
+// only while consecutive steps lay the buffer out the same way (the input
+// part of one step must not overlap the output part of the previous one), so
+// an entry holds the layout it was recorded for: a step with another graph,
+// width, dtype or staging size -- or a buffer whose entry was reused, or that
+// was never seen -- gets the full ordering after `stream` again.
 constexpr int kStagingSlots = 16;
-struct StagingOrder {
+struct StagingKey {
     const void *staging = nullptr;
     int device = -1;
+    const ag_graph *graph = nullptr;
+    int64_t N = 0, E = 0, H = 0;
+    int dtype = -1;
+    size_t bytes = 0;
+    bool operator==(const StagingKey &o) const {
+        return staging == o.staging && device == o.device && graph == o.graph && N == o.N && E == o.E &&
+               H == o.H && dtype == o.dtype && bytes == o.bytes;
+    }
+};
+struct StagingOrder {
+    StagingKey key;
     cudaEvent_t done = nullptr;
 };
 StagingOrder g_staging[kStagingSlots];
 int g_staging_next = 0;
 
-StagingOrder *find_staging(const void *staging, int device) {
+// The entry of this buffer (same address and device), whatever its layout.
+StagingOrder *find_staging(const StagingKey &k) {
     for (auto &s : g_staging)
-        if (s.done && s.staging == staging && s.device == device) return &s;
+        if (s.done && s.key.staging == k.staging && s.key.device == k.device) return &s;
     return nullptr;
 }
 
 // Make `in` wait for the previous step's reads of the staging buffer's
-// inputs (pipelined), or for everything on `st` so far (first use).
-cudaError_t staging_wait_inputs(const void *staging, int device, cudaStream_t st, cudaStream_t in, cudaEvent_t tmp) {
+// inputs (pipelined, same layout), or for everything on `st` so far (first
+// use of the buffer, or a new layout).
+cudaError_t staging_wait_inputs(const StagingKey &k, cudaStream_t st, cudaStream_t in, cudaEvent_t tmp) {
     std::lock_guard<std::mutex> lock(g_step_mu);
-    if (StagingOrder *s = find_staging(staging, device)) return cudaStreamWaitEvent(in, s->done, 0);
-    StagingOrder &s = g_staging[g_staging_next];
-    g_staging_next = (g_staging_next + 1) % kStagingSlots;
-    if (s.done) cudaEventDestroy(s.done);  // released once its pending waits are done
-    s = StagingOrder{};
-    cudaError_t err = cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming);
-    if (err != cudaSuccess) {
-        s.done = nullptr;
-        return err;
+    StagingOrder *s = find_staging(k);
+    if (s && s->key == k) return cudaStreamWaitEvent(in, s->done, 0);
+    if (!s) {
+        s = &g_staging[g_staging_next];
+        g_staging_next = (g_staging_next + 1) % kStagingSlots;
+        if (s->done) cudaEventDestroy(s->done);  // released once its pending waits are done
+        *s = StagingOrder{};
+        cudaError_t err = cudaEventCreateWithFlags(&s->done, cudaEventDisableTiming);
+        if (err != cudaSuccess) {
+            s->done = nullptr;
+            return err;
+        }
     }
-    s.staging = staging;
-    s.device = device;
-    err = cudaEventRecord(tmp, st);
+    s->key = k;  // a new layout keeps the buffer's event, ordered after `st` below
+    cudaError_t err = cudaEventRecord(tmp, st);
     return err == cudaSuccess ? cudaStreamWaitEvent(in, tmp, 0) : err;
 }
 
 // After a step's backward pass (on st): the staging buffer's inputs are read.
-cudaError_t staging_mark_read(const void *staging, int device, cudaStream_t st) {
+cudaError_t staging_mark_read(const StagingKey &k, cudaStream_t st) {
     std::lock_guard<std::mutex> lock(g_step_mu);
-    if (StagingOrder *s = find_staging(staging, device)) return cudaEventRecord(s->done, st);
+    StagingOrder *s = find_staging(k);
+    if (s && s->key == k) return cudaEventRecord(s->done, st);
     return cudaSuccess;
 }
 }  // namespace
@@ -1602,10 +2054,19 @@ int step_host(const ag_graph *g, const float *w_host, const void *X_host, const 
         if (err == cudaSuccess) err = cudaStreamWaitEvent(s, e, 0);
     };
     const size_t scr = scratch_needed(g, H);  // staging's scratch part
+    StagingKey key;
+    key.staging = staging;
+    key.device = g->device;
+    key.graph = g;
+    key.N = g->N;
+    key.E = g->E;
+    key.H = H;
+    key.dtype = dtype;
+    key.bytes = staging_bytes;
     if (pipelined) {
         // all inputs on the helper stream, after the previous step's backward
         // pass on this staging buffer (not after its copies out)
-        if (err == cudaSuccess) err = staging_wait_inputs(staging, g->device, st, s_in, ev.e[5]);
+        if (err == cudaSuccess) err = staging_wait_inputs(key, st, s_in, ev.e[5]);
         copy(w, w_host, wb, cudaMemcpyHostToDevice, s_in);
         copy(X, X_host, feat, cudaMemcpyHostToDevice, s_in);
         record(ev.e[0], s_in);
@@ -1628,7 +2089,7 @@ int step_host(const ag_graph *g, const float *w_host, const void *X_host, const 
     wait(st, ev.e[1]);
     if (err != cudaSuccess) return cuda_fail(err, fn);
     if ((rc = backward(g, w, X, dY, dX, dw, H, dtype, scratch, scr, stream, fn, false)) != AG_OK) return rc;
-    if (err == cudaSuccess) err = staging_mark_read(staging, g->device, st);
+    if (err == cudaSuccess) err = staging_mark_read(key, st);
     record(ev.e[3], st);
     wait(s_out, ev.e[3]);
     copy(dX_host, dX, feat, cudaMemcpyDeviceToHost, s_out);
