@@ -2,10 +2,12 @@
 """Throughput of the fused weighted GNN aggregation step on B200.
 
 A step is one pass of the whole per-call hot path over one batch of inputs on
-a lowered (fixed) topology: forward Y = A_w X (ag_spmm_fwd), then feature
-gradient dX = A_w^T dY and weight gradient dw_e = dot(X[src_e], dY[dst_e]) in
-one fused pass (ag_backward).  The separate ag_spmm_dx and ag_sddmm_dw entry
-points are timed after the step for the per-kernel breakdown.  The default workload is
+a lowered (fixed) topology: forward Y = A_w X, feature gradient
+dX = A_w^T dY and weight gradient dw_e = dot(X[src_e], dY[dst_e]), through
+ag_step (the forward pass and the fused backward pass of ag_backward in one
+call, the two overlapped).  ag_spmm_fwd and ag_backward, and the separate
+ag_spmm_dx and ag_sddmm_dw entry points, are timed after the step for the
+per-kernel breakdown.  The default workload is
 the R-MAT scale-22 graph (4,194,304 nodes, 67,108,864 edges, H = 128, bf16
 features with fp32 accumulation), whose inputs (X and dY are 1 GiB each) are
 larger than L2, so no flush is needed between steps.
@@ -102,10 +104,11 @@ def row_bytes(N, E, H, elem):
 
 
 def launches_per_step_of(st, wl):
-    """Kernels one step launches: ag_spmm_fwd = weight regroup + tile walk
-    (+ fixup when rows span tiles); ag_backward on the single-walk shapes (the
-    whole width in one lane group pass, as for H=128) = weight regroup + fused
-    walk (+ fixup) + dw regroup back to COO order."""
+    """Kernels one step (ag_step) launches, the same as ag_spmm_fwd followed by
+    ag_backward: forward = weight regroup + tile walk (+ fixup when rows span
+    tiles); backward on the single-walk shapes (the whole width in one lane
+    group pass, as for H=128) = weight regroup + fused walk (+ fixup) + dw
+    regroup back to COO order."""
     if wl.E == 0:
         return int(wl.N > 0) * 2
     fwd = 2 + int(st["spanning_rows_f"] > 0)
@@ -328,7 +331,8 @@ def workload_config(wl, args):
                 2 if wl.feature_dtype == torch.bfloat16 else 4) > (126 << 20) else
                   "inputs smaller than L2: warm-L2 numbers",
             "l2_persistence": "not set (no access policy window, default L2 set-aside)",
-            "step": "ag_spmm_fwd + ag_backward (dX and dw fused) on a lowered graph; value = E*H per step / step time"}
+            "step": "ag_step: forward (ag_spmm_fwd) and fused backward (ag_backward: dX and dw) in one call, "
+                    "the two passes overlapped, on a lowered graph; value = E*H per step / step time"}
 
 
 def profile_once(args):
@@ -407,23 +411,17 @@ def our_arm(args):
     g.scratch(wl.H)
 
     ops = ("fwd", "backward")
+    agb.ag_step(g, wl.w, wl.X, wl.dY, Y, dX, dw)  # allocates the step's scratch once
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        agb.ag_spmm_fwd(g, wl.w, wl.X, Y)
-        if ev is not None:
-            ev[1].record(stream)
-        agb.ag_backward(g, wl.w, wl.X, wl.dY, dX, dw)
-        if ev is not None:
-            ev[2].record(stream)
+    def step():
+        # forward + fused backward in one call (the two passes overlapped)
+        agb.ag_step(g, wl.w, wl.X, wl.dY, Y, dX, dw)
 
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -431,17 +429,17 @@ def our_arm(args):
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
         for k in range(K):
-            step(evs[k])
+            step()
         end.record(stream)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
     clocks = clk.summary()
     ms = start.elapsed_time(end)
-    per_op = {op: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)] for i, op in enumerate(ops)}
     ms = max_over_ranks(ms, dev)
 
-    # the separate gradient entry points, for the per-kernel breakdown (not in the step)
+    # the entry points of the step one by one, and the separate gradient
+    # entry points, for the per-kernel breakdown (not in the step)
     def timed(fn, reps):
         for _ in range(2):
             fn()
@@ -454,6 +452,9 @@ def our_arm(args):
         torch.cuda.synchronize()
         return [e[i].elapsed_time(e[i + 1]) for i in range(reps)]
 
+    per_op = {}
+    per_op["fwd"] = timed(lambda: agb.ag_spmm_fwd(g, wl.w, wl.X, Y), K)
+    per_op["backward"] = timed(lambda: agb.ag_backward(g, wl.w, wl.X, wl.dY, dX, dw), K)
     per_op["dx"] = timed(lambda: agb.ag_spmm_dx(g, wl.w, wl.dY, dX), K)
     per_op["dw"] = timed(lambda: agb.ag_sddmm_dw(g, wl.X, wl.dY, dw), K)
 

@@ -14,6 +14,7 @@ and "Edge order is explicit"), with A_w[dst_e, src_e] = w_e:
     ag_spmm_dx(g, w, dY)         -> dX = A_w^T dY
     ag_sddmm_dw(g, X, dY)        -> dw_e = dot(X[src_e], dY[dst_e])   (COO order)
     ag_backward(g, w, X, dY)     -> (dX, dw) in one pass over the transpose CSR
+    ag_step(g, w, X, dY)         -> (Y, dX, dw): forward and fused backward in one call, overlapped
     ag_step_host(g, w, X, dY, ...)  the three from host buffers, copies included
     ag_step_host_pipelined(...)     the same for back-to-back steps (copies overlap across steps)
 """
@@ -26,7 +27,8 @@ import re
 import torch
 
 __all__ = ["AggraphError", "Graph", "ag_graph_lower", "ag_spmm_fwd", "ag_spmm_dx", "ag_sddmm_dw", "ag_backward",
-           "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward", "ag_step_host", "ag_step_host_pipelined", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
+           "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward", "ag_step",
+           "ag_step_host", "ag_step_host_pipelined", "ag_step_staging_bytes", "ag_graph_workspace_bytes", "lib", "LIB_PATH",
            "declared_symbols", "AG_F32", "AG_BF16"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaggraph.so")
@@ -96,13 +98,17 @@ def _bind(handle: ctypes.CDLL) -> ctypes.CDLL:
     handle.ag_step_staging_bytes.restype = _SZ
     handle.ag_step_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_step_host_pipelined.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
+    handle.ag_step_scratch_bytes.argtypes = [_P, _I64]
+    handle.ag_step_scratch_bytes.restype = _SZ
+    handle.ag_step.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I, _P, _SZ, _P]
     handle.ag_graph_free.argtypes = [_P]
     handle.ag_graph_free.restype = None
     handle.ag_last_error.restype = ctypes.c_char_p
     handle.ag_status_string.argtypes = [_I]
     handle.ag_status_string.restype = ctypes.c_char_p
     for name in ("ag_graph_lower", "ag_graph_arrays", "ag_graph_get_stats", "ag_spmm_fwd", "ag_spmm_dx",
-                 "ag_sddmm_dw", "ag_backward", "ag_spmm_fwd_static_scratch", "ag_step_host", "ag_step_host_pipelined", "ag_abi_version",
+                 "ag_sddmm_dw", "ag_backward", "ag_step", "ag_spmm_fwd_static_scratch", "ag_step_host",
+                 "ag_step_host_pipelined", "ag_abi_version",
                  "ag_mean_fwd", "ag_mean_backward", "ag_gcn_norm", "ag_attn_fwd", "ag_attn_backward"):
         getattr(handle, name).restype = _I
     return handle
@@ -179,6 +185,7 @@ class Graph:
         _check(lib.ag_graph_get_stats(self._h, ctypes.byref(st)))
         self.stats = st.as_dict()
         self._scratch: dict = {}
+        self._step_scratch: dict = {}
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -321,6 +328,38 @@ def ag_backward(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, dX
     _check(lib.ag_backward(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(dX), _ptr(dw), H, code, _ptr(scr),
                            0 if scr is None else scr.numel(), _stream(g.device, stream)))
     return dX, dw
+
+
+def ag_step(g: Graph, w: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, Y=None, dX=None, dw=None,
+            stream=None):
+    """(Y, dX, dw) = (A_w X, A_w^T dY, dot(X[src_e], dY[dst_e])) in one call: the forward
+    pass and the fused backward pass, overlapped (bitwise equal to ag_spmm_fwd + ag_backward)."""
+    _check_edge_vec(g, "w", w)
+    code = _check_feat(g, "X", X)
+    if _check_feat(g, "dY", dY) != code or dY.shape != X.shape:
+        raise AggraphError(2, "X and dY must have the same shape and dtype")
+    outs = []
+    for name, t in (("Y", Y), ("dX", dX)):
+        if t is None:
+            t = torch.empty_like(X)
+        elif t.shape != X.shape or t.dtype != X.dtype:
+            raise AggraphError(2, f"{name} must match X in shape and dtype")
+        else:
+            _need_cuda(name, t)
+        outs.append(t)
+    if dw is None:
+        dw = torch.empty(g.E, dtype=torch.float32, device=g.device)
+    else:
+        _check_edge_vec(g, "dw", dw)
+    H = X.shape[1]
+    n = int(lib.ag_step_scratch_bytes(g.handle, H))
+    scr = g._step_scratch.get(H)
+    if scr is None or scr.numel() < n:
+        scr = torch.empty(max(n, 1), dtype=torch.uint8, device=g.device)
+        g._step_scratch[H] = scr
+    _check(lib.ag_step(g.handle, _ptr(w), _ptr(X), _ptr(dY), _ptr(outs[0]), _ptr(outs[1]), _ptr(dw), H, code,
+                       _ptr(scr), n, _stream(g.device, stream)))
+    return outs[0], outs[1], dw
 
 
 def ag_mean_fwd(g: Graph, w, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:

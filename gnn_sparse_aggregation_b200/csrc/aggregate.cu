@@ -1681,10 +1681,6 @@ int backward(const ag_graph *g, const float *w, const void *X, const void *dY, v
 
 // ---------------------------------------------------------------- GCN weights
 
-__global__ void k_fill(float *__restrict__ p, int64_t n, float v) {
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
-        p[i] = v;
-}
 // unit weights: the degree is the row length of the forward CSR
 __global__ void k_row_counts(const int32_t *__restrict__ rowptr, int64_t N, float *__restrict__ deg) {
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < N; i += int64_t(gridDim.x) * blockDim.x)
@@ -1696,6 +1692,17 @@ __global__ void k_inv_sqrt(float *__restrict__ deg, int64_t N) {
         const float d = deg[i];
         deg[i] = d > 0.f ? 1.f / sqrtf(d) : 0.f;
     }
+}
+// deg[i]^-1/2 from the row sums sums[i].x (rows without edges hold 0)
+__global__ void k_inv_sqrt_sums(const float2 *__restrict__ sums, int64_t N, float *__restrict__ deg) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < N; i += int64_t(gridDim.x) * blockDim.x) {
+        const float d = sums[i].x;
+        deg[i] = d > 0.f ? 1.f / sqrtf(d) : 0.f;
+    }
+}
+__global__ void k_zero2(float2 *__restrict__ p, int64_t n) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+        p[i] = make_float2(0.f, 0.f);
 }
 // out[e] = dis[src_e] * w_e * dis[dst_e] in COO order (w = null: 1)
 __global__ void k_gcn_weights(const int32_t *__restrict__ src, const int32_t *__restrict__ dst,
@@ -1711,16 +1718,18 @@ unsigned flat_grid(int64_t n) {
     return unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
 }
 
-// Scratch of ag_gcn_norm: deg[N] | ones[N] | scratch of a width-1 SpMM.
+// Scratch of ag_gcn_norm: deg[N] | row sums float2[N] | tile partials
+// float2[2 tiles] | weights in forward windows float[E].
 struct GcnLayout {
-    size_t deg, ones, spmm, total;
+    size_t deg, sums, partial, w_b, total;
 };
 GcnLayout gcn_layout(const ag_graph *g) {
     GcnLayout L;
     L.deg = 0;
-    L.ones = align_up(size_t(g->N) * 4);
-    L.spmm = L.ones + align_up(size_t(g->N) * 4);
-    L.total = L.spmm + scratch_needed(g, 1);
+    L.sums = align_up(size_t(g->N) * 4);
+    L.partial = L.sums + align_up(size_t(g->N) * 8);
+    L.w_b = L.partial + align_up(size_t(2) * size_t(g->n_tiles) * 8);
+    L.total = L.w_b + align_up(size_t(g->E) * 4);
     return L;
 }
 
@@ -1740,40 +1749,24 @@ int gcn_norm(const ag_graph *g, const float *w, float *w_norm, void *scratch, si
     char *scr = static_cast<char *>(scratch);
     float *deg = reinterpret_cast<float *>(scr + L.deg);
     if (w) {
-        // weighted in-degree = A_w 1: the forward SpMM of a column of ones
-        float *ones = reinterpret_cast<float *>(scr + L.ones);
-        k_fill<<<flat_grid(g->N), kThreads, 0, st>>>(ones, g->N, 1.f);
-        rc = spmm(g, 0, w, ones, deg, 1, AG_F32, scr + L.spmm, scratch_bytes - L.spmm, stream, fn, false);
+        // weighted in-degree: the weights summed over each forward-CSR row
+        // (a segmented reduction in a fixed order, over the weights regrouped
+        // into the forward walk's windows)
+        float *w_b = reinterpret_cast<float *>(scr + L.w_b);
+        float2 *sums = reinterpret_cast<float2 *>(scr + L.sums);
+        regroup(true, g->dir[0], w, g->E, w_b, st);
+        k_zero2<<<flat_grid(g->N), kThreads, 0, st>>>(sums, g->N);
+        rc = row_sums(g, w_b, reinterpret_cast<float2 *>(scr + L.partial), sums, st);
         if (rc != AG_OK) return rc;
+        k_inv_sqrt_sums<<<flat_grid(g->N), kThreads, 0, st>>>(sums, g->N, deg);
     } else {
         k_row_counts<<<flat_grid(g->N), kThreads, 0, st>>>(g->dir[0].rowptr, g->N, deg);
+        k_inv_sqrt<<<flat_grid(g->N), kThreads, 0, st>>>(deg, g->N);
     }
-    k_inv_sqrt<<<flat_grid(g->N), kThreads, 0, st>>>(deg, g->N);
     k_gcn_weights<<<flat_grid(g->E), kThreads, 0, st>>>(g->coo_src, g->coo_dst, w, deg, g->E, w_norm);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail(err, fn);
     return AG_OK;
-}
-
-// The SpMM walk over direction d with weights already in that direction's
-// window slots (no regrouping): out = A_w F (d = 0) or A_w^T F (d = 1).
-// scratch: an SpMM scratch of width H (its partial rows are used).
-int spmm_bucketed_impl(const ag_graph *g, int d, const float *w_b, const void *F, void *out, int64_t H, int dtype,
-                       void *scratch, cudaStream_t st) {
-    const ag::Direction &D = g->dir[d];
-    const ScratchLayout SL = scratch_layout(g, H);
-    const Shape s = pick_shape(H, dtype, F, out, nullptr);
-    Params P = base_params(g, D, H, s);
-    P.F = F;
-    P.out = out;
-    P.w = w_b;
-    P.order = D.bucket_of_pos;
-    P.partial = reinterpret_cast<float *>(static_cast<char *>(scratch) + SL.partial);
-    P.n_zero = g->N - D.n_nz;
-    if (P.n_tiles + P.n_zero > 0) dispatch_main<kSpmm>(P, s, dtype, st);
-    if (D.n_span > 0) dispatch_fixup(D, P.partial, out, H, s, dtype, st);
-    cudaError_t err = cudaGetLastError();
-    return err == cudaSuccess ? AG_OK : cuda_fail(err, "bucketed SpMM");
 }
 
 // The SDDMM walk over direction d: out_b[slot of position p] = dot(R[row of
@@ -1796,20 +1789,12 @@ int sddmm_bucketed_impl(const ag_graph *g, int d, const void *R, const void *F, 
 
 }  // namespace
 
-int spmm_bucketed(const ag_graph *g, int d, const float *w_b, const void *F, void *out, int64_t H, int dtype,
-                  void *scratch, cudaStream_t st) {
-    return spmm_bucketed_impl(g, d, w_b, F, out, H, dtype, scratch, st);
-}
 int sddmm_bucketed(const ag_graph *g, int d, const void *R, const void *F, float *out_b, int64_t H, int dtype,
                    cudaStream_t st) {
     return sddmm_bucketed_impl(g, d, R, F, out_b, H, dtype, st);
 }
 void regroup_from_buckets(const ag_graph *g, int d, const float *in_b, float *out, cudaStream_t st) {
     regroup(false, g->dir[d], in_b, g->E, out, st);
-}
-int backward_into(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw, int64_t H,
-                  int dtype, void *scratch, size_t scratch_bytes, cudaStream_t st) {
-    return backward(g, w, X, dY, dX, dw, H, dtype, scratch, scratch_bytes, st, "ag_attn_backward", false);
 }
 
 size_t spmm_scratch_edge_offset(const ag_graph *g, int64_t H, int which) {
@@ -2116,6 +2101,128 @@ int ag_step_host_pipelined(const ag_graph *g, const float *w_host, const void *X
                            size_t staging_bytes, void *stream) {
     return step_host(g, w_host, X_host, dY_host, Y_host, dX_host, dw_host, H, dtype, staging, staging_bytes,
                      stream, true, "ag_step_host_pipelined");
+}
+
+// ---------------------------------------------------------------------------- one step in one call
+
+}  // extern "C"
+
+namespace {
+// Scratch of ag_step: the backward pass's SpMM scratch, then the forward
+// pass's partial rows and its weights in forward windows.
+struct StepLayout {
+    ScratchLayout bwd;
+    size_t fwd_partial, fwd_w_b, total;
+};
+StepLayout step_layout(const ag_graph *g, int64_t H) {
+    StepLayout L;
+    L.bwd = scratch_layout(g, H);
+    const bool spans = g->dir[0].n_span > 0 || g->dir[1].n_span > 0;
+    L.fwd_partial = align_up(L.bwd.total);
+    L.fwd_w_b = L.fwd_partial + align_up(spans ? size_t(2) * size_t(g->n_tiles) * size_t(H) * 4 : 0);
+    L.total = L.fwd_w_b + align_up(size_t(g->E) * 4);
+    return L;
+}
+
+int step_device(const ag_graph *g, const float *w, const void *X, const void *dY, void *Y, void *dX, float *dw,
+                int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream) {
+    const char *fn = "ag_step";
+    int rc = check_call(g, H, dtype, fn);
+    if (rc != AG_OK) return rc;
+    if (!X || !dY || !Y || !dX || (g->E > 0 && (!w || !dw)))
+        return fail(AG_ERR_INVALID_ARG, "%s: null w, X, dY, Y, dX or dw", fn);
+    const StepLayout L = step_layout(g, H);
+    if ((rc = check_scratch(g, L.total, scratch, scratch_bytes, fn)) != AG_OK) return rc;
+    const void *ptrs[] = {X, dY, Y, dX, scratch};
+    const char *names[] = {"X", "dY", "Y", "dX", "scratch"};
+    for (int i = 0; i < 5; ++i)
+        if ((rc = check_device_ptr(ptrs[i], g->device, names[i])) != AG_OK) return rc;
+    if (g->E > 0) {
+        if ((rc = check_device_ptr(w, g->device, "w")) != AG_OK) return rc;
+        if ((rc = check_device_ptr(dw, g->device, "dw")) != AG_OK) return rc;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Shape sf = pick_shape(H, dtype, X, Y, nullptr);
+    const Shape sb = pick_shape(H, dtype, X, dY, dX);
+    if (g->E == 0 || !ring_shape(sb, dtype, H)) {
+        // shapes without the single backward walk: the two calls in order
+        rc = spmm(g, 0, w, X, Y, H, dtype, scratch, L.bwd.total, stream, fn, false);
+        if (rc == AG_OK) rc = backward(g, w, X, dY, dX, dw, H, dtype, scratch, L.bwd.total, stream, fn, false);
+        return rc;
+    }
+    cudaStream_t side = nullptr, unused = nullptr;
+    if ((rc = step_streams(g->device, &side, &unused)) != AG_OK) return rc;
+    StepEvents ev;
+    cudaError_t err = ev.create();
+    auto record = [&](cudaEvent_t e, cudaStream_t s) {
+        if (err == cudaSuccess) err = cudaEventRecord(e, s);
+    };
+    auto wait = [&](cudaStream_t s, cudaEvent_t e) {
+        if (err == cudaSuccess) err = cudaStreamWaitEvent(s, e, 0);
+    };
+    char *scr = static_cast<char *>(scratch);
+    float *w_b_f = reinterpret_cast<float *>(scr + L.fwd_w_b);
+    float *w_b_t = reinterpret_cast<float *>(scr + L.bwd.w_b);
+    float *dw_b = reinterpret_cast<float *>(scr + L.bwd.dw_b);
+    // side: the forward weights into their windows, while the backward walk runs
+    record(ev.e[0], st);
+    wait(side, ev.e[0]);
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    regroup(true, g->dir[0], w, g->E, w_b_f, side);
+    record(ev.e[1], side);
+    // main: the fused backward walk over the transpose CSR
+    const ag::Direction &Dt = g->dir[1];
+    Params Pb = base_params(g, Dt, H, sb);
+    regroup(true, Dt, w, g->E, w_b_t, st);
+    Pb.order = Dt.bucket_of_pos;
+    Pb.w = w_b_t;
+    Pb.F = dY;
+    Pb.R = X;
+    Pb.out = dX;
+    Pb.dw = dw_b;
+    Pb.partial = reinterpret_cast<float *>(scr + L.bwd.partial);
+    Pb.n_zero = g->N - Dt.n_nz;
+    dispatch_main<kBoth>(Pb, sb, dtype, st);
+    record(ev.e[2], st);
+    // side: the backward's rows cut by tiles and dw back to COO order, while
+    // the forward walk runs (the two passes use separate partial rows)
+    wait(side, ev.e[2]);
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    if (Dt.n_span > 0) dispatch_fixup(Dt, Pb.partial, dX, H, sb, dtype, side);
+    regroup(false, Dt, dw_b, g->E, dw, side);
+    record(ev.e[3], side);
+    // main: the forward walk
+    const ag::Direction &Df = g->dir[0];
+    Params Pf = base_params(g, Df, H, sf);
+    Pf.order = Df.bucket_of_pos;
+    Pf.w = w_b_f;
+    Pf.F = X;
+    Pf.out = Y;
+    Pf.partial = reinterpret_cast<float *>(scr + L.fwd_partial);
+    Pf.n_zero = g->N - Df.n_nz;
+    wait(st, ev.e[1]);
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    if (Pf.n_tiles + Pf.n_zero > 0) dispatch_main<kSpmm>(Pf, sf, dtype, st);
+    if (Df.n_span > 0) dispatch_fixup(Df, Pf.partial, Y, H, sf, dtype, st);
+    // `stream` is ordered after the side stream's work
+    wait(st, ev.e[3]);
+    if (err == cudaSuccess) err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, fn);
+    return AG_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t ag_step_scratch_bytes(const ag_graph *g, int64_t H) {
+    if (!g || H < 1) return 0;
+    return step_layout(g, H).total;
+}
+
+int ag_step(const ag_graph *g, const float *w, const void *X, const void *dY, void *Y, void *dX, float *dw, int64_t H,
+            int dtype, void *scratch, size_t scratch_bytes, void *stream) {
+    clear_error();
+    return step_device(g, w, X, dY, Y, dX, dw, H, dtype, scratch, scratch_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------- forward without caller scratch

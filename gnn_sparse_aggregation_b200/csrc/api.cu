@@ -172,6 +172,6 @@ const char *ag_status_string(int status) {
     }
 }
 
-int ag_abi_version(void) { return 101; }  // 1.01: ag_step_host_pipelined added
+int ag_abi_version(void) { return 102; }  // 1.02: ag_step added
 
 }  // extern "C"

@@ -7,23 +7,18 @@
 //   alpha_e = exp(s_e - m_r) / l_r,  r = dst_e           (row softmax)
 //   Y[r]    = sum over edges e into r of alpha_e V[src_e] (SpMM)
 //
-// The scores and the SpMMs run on this library's own walks.  Per-edge values
-// stay in the window slots of the walk that made or reads them wherever
-// possible: the forward pass computes the scores with the SDDMM walk of the
-// forward CSR straight into its window slots, reduces them per row there,
-// writes alpha into the same slots (the aggregation reads them unmoved) and
-// moves alpha once, back to COO order, for the caller.  The backward pass
-// takes dV and dalpha from one transpose walk (ag_backward with weights
-// alpha and "features" V), which leaves alpha and dalpha in the transpose
-// walk's slots; c_r = sum of alpha dalpha per row is reduced from copies in
-// the forward walk's slots; ds is formed in both walks' slots, and dQ and dK
-// are the two SpMMs of ds without further regrouping.  The row statistics
-// m_r (maximum) and l_r (sum of exp(s - m_r)) come from one segmented
-// reduction over the forward CSR, walked in the same edge-balanced tiles as
-// the SpMM: one warp per tile, Hillis-Steele segmented scans per 32
-// positions, rows cut by a tile boundary finished by a fixup pass in tile
-// order.  Every reduction tree is fixed by the positions alone, so results
-// are deterministic.
+// The scores come from the SDDMM walk of the forward CSR (owner Q[dst],
+// gathered K[src]) straight into the forward walk's window slots, where the
+// row statistics read them; they then go back to COO order once, for the
+// softmax.  The SpMMs run through this library's own entry points
+// (ag_spmm_fwd, ag_spmm_dx, and ag_backward for dV with dalpha in one walk);
+// the per-edge inputs of the backward's row reduction are first regrouped
+// into the forward walk's window-bucketed order; the row statistics m_r (maximum)
+// and l_r (sum of exp(s - m_r)) come from one segmented reduction over the
+// forward CSR, walked in the same edge-balanced tiles as the SpMM: one warp
+// per tile, Hillis-Steele segmented scans per 32 positions, rows cut by a
+// tile boundary finished by a fixup pass in tile order.  Every reduction tree
+// is fixed by the positions alone, so results are deterministic.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -73,10 +68,11 @@ __device__ __forceinline__ float2 shfl2(float2 v, int src) {
     return make_float2(__shfl_sync(kFull, v.x, src), __shfl_sync(kFull, v.y, src));
 }
 
-// Leaf value of COO edge e: kSoftmaxStats the score scale * a_e, kSum a_e * b_e.
+// Leaf value of COO edge e: kSoftmaxStats the score scale * a_e, kSum a_e * b_e
+// (a_e alone when there is no b).
 template <int OP>
 __device__ __forceinline__ float leaf_value(const ReduceParams &P, int e) {
-    return OP == kSoftmaxStats ? P.scale * P.a[e] : P.a[e] * P.b[e];
+    return OP == kSoftmaxStats ? P.scale * P.a[e] : (P.b ? P.a[e] * P.b[e] : P.a[e]);
 }
 
 // Segmented inclusive scan over the 32 lanes (segment of lane i: from its
@@ -103,18 +99,30 @@ constexpr int kMaxChunks = kMaxTileEdges / 32;
 
 template <int OP>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const ReduceParams P) {
+    // the first positions of the rows after the open one, up to the last row
+    // that starts in the tile (at most T of them), staged per warp so that the
+    // chunk-to-chunk chain below waits on shared memory, not on global loads
+    __shared__ int row_start[kWarpsPerBlock][kMaxTileEdges + 1];
     const int64_t t = (int64_t(blockIdx.x) * kWarpsPerBlock) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (t >= P.n_tiles) return;  // whole warps
+    int *rs = row_start[threadIdx.x >> 5];
     const int64_t p0 = t * P.T;
     const int len = int(P.E - p0 < P.T ? P.E - p0 : P.T);
     float x[kMaxChunks];
     int e[kMaxChunks];
 #pragma unroll
     for (int c = 0; c < kMaxChunks; ++c) e[c] = c * 32 + lane < len ? __ldcs(P.order + p0 + c * 32 + lane) : -1;
+    const int64_t r0 = P.tile_nz[t];
+    // rows r0 + 1 .. r_last: the row holding the next tile's first position
+    // closes the range (the last tile: the last row)
+    const int64_t r_last = t + 1 < P.n_tiles ? P.tile_nz[t + 1] : P.n_nz - 1;
+    const int nrs = int(r_last - r0);  // <= T: at most one row starts per position
+    for (int i = lane; i < nrs; i += 32) rs[i] = P.nz_rowptr[r0 + 1 + i];
 #pragma unroll
     for (int c = 0; c < kMaxChunks; ++c) x[c] = e[c] >= 0 ? leaf_value<OP>(P, e[c]) : 0.f;
-    int64_t cur = P.tile_nz[t];
+    __syncwarp();
+    int64_t cur = r0;
     bool before = P.nz_rowptr[cur] < p0;
     float2 acc = identity<OP>();
 #pragma unroll
@@ -125,9 +133,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const Reduce
         const int n = len - base < 32 ? len - base : 32;
         // starts of the rows after the open one that fall inside the chunk
         unsigned bit = 0;
-        const int64_t k = cur + 1 + lane;
-        if (k < P.n_nz) {
-            const int64_t st = P.nz_rowptr[k];
+        const int64_t k = cur + 1 + lane - (r0 + 1);  // index into the staged row starts
+        if (k < nrs) {
+            const int64_t st = rs[k];
             if (st >= cb && st < cb + n) bit = 1u << int(st - cb);
         }
         const unsigned mask = __reduce_or_sync(kFull, bit);
@@ -185,53 +193,20 @@ __global__ void k_row_reduce_fixup(const int4 *__restrict__ spans, int64_t n_spa
     out[sp.x] = v;
 }
 
-enum PositionOp { kAlpha = 0, kDs = 1 };
-
-// Per forward-CSR position p of row r, in the forward walk's window slots
-// (slot = order[p]), one warp per tile walking 32 positions at a time (each
-// lane's row is found from the chunk's row-start mask, as in k_row_reduce):
-//   kAlpha: out[slot] = expf(scale * a[slot] - m_r) / l_r      (stats = (m, l))
-//   kDs   : out[slot] = scale * a[slot] * (b[slot] - c_r)      (stats = (c, 0); in place over b)
-template <int OP>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
-k_per_position(const ReduceParams P, const float2 *__restrict__ stats, float *out) {
-    const int64_t t = (int64_t(blockIdx.x) * kWarpsPerBlock) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (t >= P.n_tiles) return;  // whole warps
-    const int64_t p0 = t * P.T;
-    const int len = int(P.E - p0 < P.T ? P.E - p0 : P.T);
-    int64_t cur = P.tile_nz[t];
-    for (int base = 0; base < len; base += 32) {
-        const int64_t cb = p0 + base;
-        const int n = len - base < 32 ? len - base : 32;
-        unsigned bit = 0;
-        const int64_t k = cur + 1 + lane;
-        if (k < P.n_nz) {
-            const int64_t st = P.nz_rowptr[k];
-            if (st >= cb && st < cb + n) bit = 1u << int(st - cb);
-        }
-        const unsigned mask = __reduce_or_sync(kFull, bit);
-        if (lane < n) {
-            const int r = P.nz_rows[cur + __popc(mask & (kFull >> (31 - lane)))];
-            const float2 s2 = stats[r];
-            const int slot = __ldcs(P.order + cb + lane);
-            if (OP == kAlpha) out[slot] = expf(P.scale * P.a[slot] - s2.x) / s2.y;
-            else out[slot] = P.scale * P.a[slot] * (P.b[slot] - s2.x);
-        }
-        cur += __popc(mask);
+// alpha_e = exp(scale * s_e - m_r) / l_r (in place over s)
+__global__ void k_softmax_alpha(float *__restrict__ s, const int32_t *__restrict__ dst, const float2 *__restrict__ ml,
+                                float scale, int64_t E) {
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
+        const float2 r = ml[__ldcs(dst + e)];
+        s[e] = expf(scale * s[e] - r.x) / r.y;
     }
 }
 
-// ds at every transpose-CSR position p, in the transpose walk's window slots
-// (in place over d_t): d_t[slot] = scale * a_t[slot] * (d_t[slot] - c[dst]),
-// dst = col_t[p]
-__global__ void k_ds_transpose(const int32_t *__restrict__ slot_of_pos, const int32_t *__restrict__ col_t,
-                               const float *__restrict__ a_t, float *d_t, const float2 *__restrict__ c, float scale,
-                               int64_t E) {
-    for (int64_t p = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; p < E; p += int64_t(gridDim.x) * blockDim.x) {
-        const int slot = __ldcs(slot_of_pos + p);
-        d_t[slot] = scale * a_t[slot] * (d_t[slot] - c[__ldcs(col_t + p)].x);
-    }
+// ds_e = scale * alpha_e * (dalpha_e - c_r) (in place over dalpha)
+__global__ void k_attn_ds(const float *__restrict__ alpha, float *__restrict__ da, const int32_t *__restrict__ dst,
+                          const float2 *__restrict__ c, float scale, int64_t E) {
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x)
+        da[e] = scale * alpha[e] * (da[e] - c[__ldcs(dst + e)].x);
 }
 
 unsigned flat_blocks(int64_t n) {
@@ -239,9 +214,9 @@ unsigned flat_blocks(int64_t n) {
     return unsigned(b < 1 ? 1 : (b > 148 * 32 ? 148 * 32 : b));
 }
 
-// scratch: SpMM scratch | per-row float2 [N] | tile partials float2 [2 tiles] | three float [E]
+// scratch: SpMM scratch | per-row float2 [N] | tile partials float2 [2 tiles] | float [E]
 struct AttnLayout {
-    size_t spmm, rows, partial, edges, edges2, edges3, total;
+    size_t spmm, rows, partial, edges, total;
 };
 AttnLayout attn_layout(const ag_graph *g, int64_t H) {
     AttnLayout L;
@@ -249,31 +224,9 @@ AttnLayout attn_layout(const ag_graph *g, int64_t H) {
     L.rows = align_up(ag_spmm_scratch_bytes(g, H));
     L.partial = L.rows + align_up(size_t(g->N) * sizeof(float2));
     L.edges = L.partial + align_up(size_t(2) * size_t(g->n_tiles) * sizeof(float2));
-    L.edges2 = L.edges + align_up(size_t(g->E) * 4);
-    L.edges3 = L.edges2 + align_up(size_t(g->E) * 4);
-    L.total = L.edges3 + align_up(size_t(g->E) * 4);
+    L.total = L.edges + align_up(size_t(g->E) * 4);
     return L;
 }
-
-ReduceParams forward_positions(const ag_graph *g, const float *a, const float *b, float scale) {
-    const Direction &D = g->dir[0];
-    ReduceParams P;
-    P.order = D.bucket_of_pos;
-    P.a = a;
-    P.b = b;
-    P.scale = scale;
-    P.T = g->tile_edges;
-    P.E = g->E;
-    P.n_tiles = g->n_tiles;
-    P.n_nz = D.n_nz;
-    P.tile_nz = D.tile_nz;
-    P.nz_rows = D.nz_rows;
-    P.nz_rowptr = D.nz_rowptr;
-    P.partial = nullptr;
-    P.out = nullptr;
-    return P;
-}
-unsigned tile_blocks(const ag_graph *g) { return unsigned((g->n_tiles + kWarpsPerBlock - 1) / kWarpsPerBlock); }
 
 // a_b, b_b: per-edge inputs already regrouped into the forward walk's
 // window-bucketed order, so that the walk's reads stay inside L2-sized
@@ -305,6 +258,17 @@ int row_reduce(const ag_graph *g, const float *a_b, const float *b_b, float scal
     cudaError_t err = cudaGetLastError();
     return err == cudaSuccess ? AG_OK : cuda_fail(err, "row reduction");
 }
+
+}  // namespace
+
+// out[r].x = sum of a_b over the forward-CSR positions of every row r with
+// edges (a_b in the forward walk's window slots); rows without edges are not
+// written.  partial: float2 [2 * tiles].
+int row_sums(const ag_graph *g, const float *a_b, float2 *partial, float2 *out, cudaStream_t st) {
+    return row_reduce<kSum>(g, a_b, nullptr, 1.f, partial, out, st);
+}
+
+namespace {
 
 int check_common(const ag_graph *g, int64_t H, int dtype, const void *scratch, size_t scratch_bytes, const char *fn,
                  AttnLayout *L) {
@@ -344,23 +308,22 @@ int ag_attn_fwd(const ag_graph *g, const void *Q, const void *K, const void *V, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *scr = static_cast<char *>(scratch);
     const size_t spmm_bytes = L.rows - L.spmm;
-    if (g->E == 0) return ag_spmm_fwd(g, alpha, V, Y, H, dtype, scr + L.spmm, spmm_bytes, stream);
-    // raw scores dot(Q[dst], K[src]) by the SDDMM walk of the forward CSR,
-    // straight into its window slots; the row statistics; alpha in the same
-    // slots; alpha back to COO order (the output) and, unmoved, the weights
-    // of the aggregation Y = A_alpha V
-    float *s_b = reinterpret_cast<float *>(scr + L.edges);
-    float *a_b = reinterpret_cast<float *>(scr + L.edges2);
-    float2 *ml = reinterpret_cast<float2 *>(scr + L.rows);
-    if ((rc = sddmm_bucketed(g, 0, Q, K, s_b, H, dtype, st)) != AG_OK) return rc;
-    rc = row_reduce<kSoftmaxStats>(g, s_b, nullptr, scale, reinterpret_cast<float2 *>(scr + L.partial), ml, st);
-    if (rc != AG_OK) return rc;
-    k_per_position<kAlpha><<<tile_blocks(g), kWarpsPerBlock * 32, 0, st>>>(forward_positions(g, s_b, nullptr, scale),
-                                                                          ml, a_b);
-    regroup_from_buckets(g, 0, a_b, alpha, st);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return cuda_fail(err, fn);
-    return spmm_bucketed(g, 0, a_b, V, Y, H, dtype, scr + L.spmm, st);
+    if (g->E > 0) {
+        // raw scores dot(Q[dst], K[src]) by the SDDMM walk of the forward CSR,
+        // straight into the forward walk's window slots (the SpMM scratch's
+        // weight-gradient array is free until the aggregation below)
+        float *s_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 1));
+        if ((rc = sddmm_bucketed(g, 0, Q, K, s_b, H, dtype, st)) != AG_OK) return rc;
+        float2 *ml = reinterpret_cast<float2 *>(scr + L.rows);
+        rc = row_reduce<kSoftmaxStats>(g, s_b, nullptr, scale, reinterpret_cast<float2 *>(scr + L.partial), ml, st);
+        if (rc != AG_OK) return rc;
+        // the scores to COO order (into alpha), then alpha in place
+        regroup_from_buckets(g, 0, s_b, alpha, st);
+        k_softmax_alpha<<<flat_blocks(g->E), 256, 0, st>>>(alpha, g->coo_dst, ml, scale, g->E);
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return cuda_fail(err, fn);
+    }
+    return ag_spmm_fwd(g, alpha, V, Y, H, dtype, scr + L.spmm, spmm_bytes, stream);
 }
 
 int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, const void *V, float scale, const float *alpha,
@@ -378,38 +341,29 @@ int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, const void
     char *scr = static_cast<char *>(scratch);
     const size_t spmm_bytes = L.rows - L.spmm;
     void *sp = scr + L.spmm;
+    float *ds = reinterpret_cast<float *>(scr + L.edges);
     if (g->E == 0) {
         if ((rc = ag_spmm_dx(g, alpha, dY, dV, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
-        if ((rc = ag_spmm_fwd(g, nullptr, K, dQ, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
-        return ag_spmm_dx(g, nullptr, Q, dK, H, dtype, sp, spmm_bytes, stream);
+    } else {
+        // dV = A_alpha^T dY and dalpha_e = dot(V[src], dY[dst]) in one transpose
+        // walk (the weighted-sum backward with weights alpha and "features" V)
+        if ((rc = ag_backward(g, alpha, V, dY, dV, ds, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+        // c_r = sum over r's edges of alpha dalpha, from bucket-ordered copies
+        // (the SpMM scratch's two per-edge arrays are free between the walks)
+        float2 *c = reinterpret_cast<float2 *>(scr + L.rows);
+        float *a_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 0));
+        float *d_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 1));
+        regroup_to_buckets(g, 0, alpha, a_b, st);
+        regroup_to_buckets(g, 0, ds, d_b, st);
+        rc = row_reduce<kSum>(g, a_b, d_b, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
+        if (rc != AG_OK) return rc;
+        k_attn_ds<<<flat_blocks(g->E), 256, 0, st>>>(alpha, ds, g->coo_dst, c, scale, g->E);
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return cuda_fail(err, fn);
     }
-    // dV = A_alpha^T dY and dalpha_e = dot(V[src], dY[dst]) in one transpose
-    // walk (the weighted-sum backward with weights alpha and "features" V);
-    // it leaves alpha and dalpha in the transpose walk's window slots, in the
-    // SpMM scratch's two per-edge arrays
-    float *da = reinterpret_cast<float *>(scr + L.edges);
-    if ((rc = backward_into(g, alpha, V, dY, dV, da, H, dtype, sp, spmm_bytes, st)) != AG_OK) return rc;
-    const float *a_t = reinterpret_cast<const float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 0));
-    float *d_t = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 1));
-    // c_r = sum over r's edges of alpha dalpha, from copies in the forward
-    // walk's window slots
-    float *a_f = reinterpret_cast<float *>(scr + L.edges2);
-    float *d_f = reinterpret_cast<float *>(scr + L.edges3);
-    float2 *c = reinterpret_cast<float2 *>(scr + L.rows);
-    regroup_to_buckets(g, 0, alpha, a_f, st);
-    regroup_to_buckets(g, 0, da, d_f, st);
-    rc = row_reduce<kSum>(g, a_f, d_f, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
-    if (rc != AG_OK) return rc;
-    // ds = scale * alpha * (dalpha - c_dst) in the slots of both walks (in place)
-    k_per_position<kDs><<<tile_blocks(g), kWarpsPerBlock * 32, 0, st>>>(forward_positions(g, a_f, d_f, scale), c,
-                                                                       d_f);
-    k_ds_transpose<<<flat_blocks(g->E), 256, 0, st>>>(g->dir[1].bucket_of_pos, g->dir[1].col, a_t, d_t, c, scale,
-                                                      g->E);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return cuda_fail(err, fn);
-    // dQ = A_ds K (scale folded into ds), dK = A_ds^T Q, from the slotted ds
-    if ((rc = spmm_bucketed(g, 0, d_f, K, dQ, H, dtype, sp, st)) != AG_OK) return rc;
-    return spmm_bucketed(g, 1, d_t, Q, dK, H, dtype, sp, st);
+    // dQ = A_ds K (scale folded into ds), dK = A_ds^T Q
+    if ((rc = ag_spmm_fwd(g, g->E > 0 ? ds : nullptr, K, dQ, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
+    return ag_spmm_dx(g, g->E > 0 ? ds : nullptr, Q, dK, H, dtype, sp, spmm_bytes, stream);
 }
 
 }  // extern "C"

@@ -110,17 +110,13 @@ size_t spmm_scratch_edge_offset(const ag_graph *g, int64_t H, int which);
 void regroup_to_buckets(const ag_graph *g, int d, const float *in, float *out_b, cudaStream_t st);
 // out[e] = in_b[bucket slot of COO edge e]: back to COO order.
 void regroup_from_buckets(const ag_graph *g, int d, const float *in_b, float *out, cudaStream_t st);
-// The SpMM of direction d (0: A_w F, 1: A_w^T F) with weights already in that
-// direction's window slots; scratch is an SpMM scratch of width H.
-int spmm_bucketed(const ag_graph *g, int d, const float *w_b, const void *F, void *out, int64_t H, int dtype,
-                  void *scratch, cudaStream_t st);
+// out[r].x = sum of a_b over the forward-CSR positions of every row r with
+// edges (a_b in the forward walk's window slots), in a fixed order; rows
+// without edges are not written.  partial: float2 [2 * tiles].
+int row_sums(const ag_graph *g, const float *a_b, float2 *partial, float2 *out, cudaStream_t st);
 // The SDDMM of direction d: out_b[slot of CSR position p] = dot(R[row of p], F[col[p]]).
 int sddmm_bucketed(const ag_graph *g, int d, const void *R, const void *F, float *out_b, int64_t H, int dtype,
                    cudaStream_t st);
-// ag_backward without the argument checks (the caller checked them); leaves
-// the weights and the weight gradient of the transpose walk in the SpMM
-// scratch's two per-edge arrays (window slots of direction 1).
-int backward_into(const ag_graph *g, const float *w, const void *X, const void *dY, void *dX, float *dw, int64_t H,
-                  int dtype, void *scratch, size_t scratch_bytes, cudaStream_t st);
+
 
 }  // namespace ag

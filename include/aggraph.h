@@ -215,6 +215,28 @@ AG_API int ag_backward(const ag_graph *g, const float *w, const void *X, const v
                        int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream);
 
 /*
+ * One training step in one call: the forward pass Y = A_w X and the fused
+ * backward pass dX = A_w^T dY, dw_e = dot(X[src_e], dY[dst_e]) (the
+ * definitions of "Edge order is explicit"; the packaging is this library's).
+ * Y, dX and dw are bitwise identical to ag_spmm_fwd followed by ag_backward.
+ * The two passes depend only on the inputs, so the call overlaps them: the
+ * backward walk runs first on `stream` while a helper stream of the device
+ * (created on first use, kept until exit) regroups the forward weights; the
+ * backward pass's rows cut by tiles and its dw regrouping then run on the
+ * helper stream while the forward walk runs on `stream`.  `stream` is
+ * ordered after all of it when the call's work is done.
+ *
+ *   w, X, dY, Y, dX, dw  as ag_spmm_fwd and ag_backward (device pointers)
+ *   scratch  device buffer of ag_step_scratch_bytes(g, H) bytes, 256-byte
+ *            aligned: ag_spmm_scratch_bytes(g, H) plus a second set of
+ *            partial rows and a second float [E] for the forward pass
+ * Errors as ag_backward; AG_ERR_CUDA also when an event cannot be created.
+ */
+AG_API size_t ag_step_scratch_bytes(const ag_graph *g, int64_t H);
+AG_API int ag_step(const ag_graph *g, const float *w, const void *X, const void *dY, void *Y, void *dX, float *dw,
+                   int64_t H, int dtype, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
  * Mean aggregation (PyTorch Geometric reading guide, Step 3: the sum and mean
  * reductions of spmm; "Done when": sum and mean are the reductions that keep
  * the semiring structure):
@@ -256,14 +278,16 @@ AG_API int ag_mean_backward(const ag_graph *g, const float *w, const void *X, co
  *   w_norm[e] = deg(src_e)^-1/2 * w_e * deg(dst_e)^-1/2, COO order,
  * with deg^-1/2 = 0 where deg <= 0.  Self-loops are whatever the edge list
  * holds (add them to the COO before lowering for the usual GCN operator).
- * The weighted degree is the forward SpMM of a column of ones (deterministic
- * order); deg^-1/2 is 1 / sqrtf(deg), both IEEE-rounded.  Feed w_norm to
+ * The weighted degree is a segmented fp32 sum of the weights over each
+ * forward-CSR row, in an order fixed by the CSR alone (deterministic);
+ * deg^-1/2 is 1 / sqrtf(deg), both IEEE-rounded.  Feed w_norm to
  * ag_spmm_fwd / ag_backward.
  *
  *   w        device float [E] (COO order) or NULL
  *   w_norm   device float [E], written (may be NULL when E == 0)
  *   scratch  device buffer, 256-byte aligned, of ag_gcn_norm_scratch_bytes(g)
- *            bytes (degrees, a column of ones and a width-1 SpMM's scratch)
+ *            bytes (degrees, row sums, per-tile partial sums and the weights
+ *            regrouped into the forward CSR's windows)
  * Errors: AG_ERR_INVALID_ARG (null graph or w_norm), AG_ERR_WORKSPACE
  * (scratch too small or misaligned), AG_ERR_DEVICE, AG_ERR_CUDA.
  */

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(agb):
 
 
 def test_status_strings_and_version(agb):
-    assert agb.lib.ag_abi_version() == 101
+    assert agb.lib.ag_abi_version() == 102
     for code, name in agb._STATUS.items():
         assert agb.lib.ag_status_string(code).decode() == name
 

@@ -13,6 +13,7 @@ import torch
 
 import workloads
 from tests.gpu_helpers import TOL, TOL_DW, assert_within, check_full, check_lowering, host, lib, run_path
+from tests.gpu_helpers import oracle_full as oracle_full_of
 from tests.golden import load
 
 pytestmark = pytest.mark.gpu
@@ -403,6 +404,37 @@ def test_pipelined_steps_with_a_new_layout_on_the_same_buffer(agb):
         assert torch.equal(bits(hY), bits(Y)), k
         assert torch.equal(bits(hdX), bits(dX)), k
         assert torch.equal(hdw, dw), k
+
+
+@pytest.mark.parametrize("case", ["uniform", "sbm", "rmat16", "twohop", "narrow-H20", "bf16-H128", "empty"])
+def test_step_equals_forward_then_backward(agb, case):
+    """ag_step (forward and fused backward in one call, the two overlapped on
+    two streams) returns exactly what ag_spmm_fwd followed by ag_backward
+    returns, on the shapes of the single backward walk and on the others
+    (which take the two calls in order), and twice in a row on one scratch."""
+    if case in ("uniform", "sbm", "rmat16", "twohop"):
+        wl = workloads.make(case, seed=4, device=DEV)
+    elif case == "empty":
+        wl = workloads.custom(50, [], [], 32, seed=4, device=DEV)
+    else:
+        N, src, dst = skewed_edges(N=2000, E=30000)
+        H, dt = (20, torch.float32) if case == "narrow-H20" else (128, torch.bfloat16)
+        wl = workloads.custom(N, src, dst, H, seed=4, feature_dtype=dt, device=DEV)
+    g = agb.ag_graph_lower(wl.src, wl.dst, wl.N)
+    ref_Y = g.fwd(wl.w, wl.X)
+    ref_dX, ref_dw = g.backward(wl.w, wl.X, wl.dY)
+    bits = (lambda t: t.view(torch.int16)) if wl.X.dtype == torch.bfloat16 else (lambda t: t.view(torch.int32))
+    for _ in range(2):
+        Y, dX, dw = agb.ag_step(g, wl.w, wl.X, wl.dY)
+        torch.cuda.synchronize()
+        assert torch.equal(bits(Y), bits(ref_Y))
+        assert torch.equal(bits(dX), bits(ref_dX))
+        assert torch.equal(dw, ref_dw)
+    if case == "rmat16":
+        (rY, bY), (rX, bX), (rw, bw) = oracle_full_of(wl)
+        assert_within(Y, rY, bY, TOL[wl.feature_dtype], "step fwd")
+        assert_within(dX, rX, bX, TOL[wl.feature_dtype], "step dX")
+        assert_within(dw, rw, bw, TOL_DW, "step dw")
 
 
 def test_errors_are_reported_not_launched(agb):
