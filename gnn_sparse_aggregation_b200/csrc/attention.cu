@@ -16,8 +16,9 @@
 // into the forward walk's window-bucketed order; the row statistics m_r (maximum)
 // and l_r (sum of exp(s - m_r)) come from one segmented reduction over the
 // forward CSR, walked in the same edge-balanced tiles as the SpMM: one warp
-// per tile, Hillis-Steele segmented scans per 32 positions, rows cut by a
-// tile boundary finished by a fixup pass in tile order.  Every reduction tree
+// per tile, each lane reducing its own run of consecutive positions in
+// registers, one Hillis-Steele segmented scan over the 32 lanes' open rows,
+// rows cut by a tile boundary finished by a fixup pass in tile order.  Every reduction tree
 // is fixed by the positions alone, so results are deterministic.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -64,8 +65,25 @@ struct ReduceParams {
     float2 *out;               // [N] per row
 };
 
-__device__ __forceinline__ float2 shfl2(float2 v, int src) {
-    return make_float2(__shfl_sync(kFull, v.x, src), __shfl_sync(kFull, v.y, src));
+__device__ __forceinline__ float2 shfl2_up(float2 v, int d) {
+    return make_float2(__shfl_up_sync(kFull, v.x, d), __shfl_up_sync(kFull, v.y, d));
+}
+
+// Adds one leaf value to a segment's aggregate: kSoftmaxStats keeps the
+// maximum m and the sum l of exp(s - m), rescaling l when m grows (one
+// exponential per value; (-inf, 0) is the empty segment); kSum adds.
+template <int OP>
+__device__ __forceinline__ void absorb(float2 &run, float s) {
+    if (OP == kSoftmaxStats) {
+        if (s > run.x) {
+            run.y = run.y * expf(run.x - s) + 1.f;
+            run.x = s;
+        } else {
+            run.y += expf(s - run.x);
+        }
+    } else {
+        run.x += s;
+    }
 }
 
 // Leaf value of COO edge e: kSoftmaxStats the score scale * a_e, kSum a_e * b_e
@@ -75,33 +93,23 @@ __device__ __forceinline__ float leaf_value(const ReduceParams &P, int e) {
     return OP == kSoftmaxStats ? P.scale * P.a[e] : (P.b ? P.a[e] * P.b[e] : P.a[e]);
 }
 
-// Segmented inclusive scan over the 32 lanes (segment of lane i: from its
-// head hs to i): op is max or sum; hs = -1 for the segment that continues
-// the open row.
-template <bool MAX>
-__device__ __forceinline__ float seg_scan(float v, int lane, int hs) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float o = __shfl_up_sync(kFull, v, off);
-        if (lane >= off && lane - off >= hs) v = MAX ? fmaxf(v, o) : v + o;
-    }
-    return v;
-}
-
-// One warp per tile of T consecutive forward-CSR positions.  All leaves of
-// the tile are loaded first (the order map, then the gathered values, two
-// round trips per tile).  Within each chunk of 32 positions the row starts
-// form a lane mask; kSoftmaxStats takes a segmented maximum M per segment,
-// one exp(s - M) per lane and a segmented sum, so every segment's (M, l)
-// sits at its last lane; kSum takes one segmented sum.  The open row (nz
-// index `cur`) carries its aggregate `acc` across chunks.
-constexpr int kMaxChunks = kMaxTileEdges / 32;
+// One warp per tile of T consecutive forward-CSR positions.  Lane l owns the
+// T / 32 consecutive positions [l T/32, (l + 1) T/32) of the tile and reduces
+// them in order in registers: every row that starts and ends inside the lane
+// is finished there; the lane's head (the positions before its first row
+// start) and its tail (the row open at its end) are combined across lanes
+// with one segmented scan over the 32 tails.  The tile's row starts are
+// staged in shared memory first; a lane finds its first row by a binary
+// search there.  kSoftmaxStats keeps (max, sum of exp(s - max)) per segment,
+// rescaling the sum when the maximum grows; kSum keeps a sum.  All leaves are
+// loaded before the reduction (the order map, then the values: two round
+// trips per tile).  Every combination order is fixed by the positions alone.
+constexpr int kMaxChunks = kMaxTileEdges / 32;  // positions per lane at most
 
 template <int OP>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const ReduceParams P) {
-    // the first positions of the rows after the open one, up to the last row
-    // that starts in the tile (at most T of them), staged per warp so that the
-    // chunk-to-chunk chain below waits on shared memory, not on global loads
+    // the first positions of the rows after the tile's first row, up to the
+    // last row that starts in the tile (at most T of them)
     __shared__ int row_start[kWarpsPerBlock][kMaxTileEdges + 1];
     const int64_t t = (int64_t(blockIdx.x) * kWarpsPerBlock) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -109,74 +117,86 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const Reduce
     int *rs = row_start[threadIdx.x >> 5];
     const int64_t p0 = t * P.T;
     const int len = int(P.E - p0 < P.T ? P.E - p0 : P.T);
-    float x[kMaxChunks];
+    const int ppl = P.T / 32;  // positions per lane (T is a power of two >= 32)
+    const int a0 = lane * ppl;
     int e[kMaxChunks];
+    float x[kMaxChunks];
 #pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c) e[c] = c * 32 + lane < len ? __ldcs(P.order + p0 + c * 32 + lane) : -1;
+    for (int k = 0; k < kMaxChunks; ++k) e[k] = (k < ppl && a0 + k < len) ? __ldg(P.order + p0 + a0 + k) : -1;
     const int64_t r0 = P.tile_nz[t];
     // rows r0 + 1 .. r_last: the row holding the next tile's first position
     // closes the range (the last tile: the last row)
     const int64_t r_last = t + 1 < P.n_tiles ? P.tile_nz[t + 1] : P.n_nz - 1;
     const int nrs = int(r_last - r0);  // <= T: at most one row starts per position
     for (int i = lane; i < nrs; i += 32) rs[i] = P.nz_rowptr[r0 + 1 + i];
+    const int64_t first_start = P.nz_rowptr[r0];  // start of the tile's first row
+    const bool before = first_start < p0;
 #pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c) x[c] = e[c] >= 0 ? leaf_value<OP>(P, e[c]) : 0.f;
+    for (int k = 0; k < kMaxChunks; ++k) x[k] = e[k] >= 0 ? leaf_value<OP>(P, e[k]) : 0.f;
     __syncwarp();
-    int64_t cur = r0;
-    bool before = P.nz_rowptr[cur] < p0;
-    float2 acc = identity<OP>();
+
+    // the row holding this lane's first position: r0 + the number of staged
+    // starts at or before it
+    const bool has_pos = a0 < len;
+    int lo = 0, hi = nrs;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (rs[mid] <= p0 + a0) lo = mid + 1;
+        else hi = mid;
+    }
+    const int64_t row_a0 = r0 + lo;
+    const bool starts_first = has_pos && (lo == 0 ? first_start : int64_t(rs[lo - 1])) == p0 + a0;
+    int64_t row_i = row_a0;
+    int64_t next = lo < nrs ? int64_t(rs[lo]) : INT64_MAX;  // start of row row_i + 1
+    bool inner = false;                                        // a row starts after the first position
+    float2 head = identity<OP>(), run = identity<OP>();
 #pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c) {
-        const int base = c * 32;
-        if (base >= len) break;  // warp-uniform
-        const int64_t cb = p0 + base;
-        const int n = len - base < 32 ? len - base : 32;
-        // starts of the rows after the open one that fall inside the chunk
-        unsigned bit = 0;
-        const int64_t k = cur + 1 + lane - (r0 + 1);  // index into the staged row starts
-        if (k < nrs) {
-            const int64_t st = rs[k];
-            if (st >= cb && st < cb + n) bit = 1u << int(st - cb);
+    for (int k = 0; k < kMaxChunks; ++k) {
+        if (k >= ppl || a0 + k >= len) break;
+        if (p0 + a0 + k == next) {  // a row starts here: close the open segment
+            if (!inner && !starts_first) head = run;
+            else P.out[P.nz_rows[row_i]] = run;  // started and ended in this lane
+            inner = true;
+            run = identity<OP>();
+            ++row_i;
+            const int m = int(row_i - r0);
+            next = m < nrs ? int64_t(rs[m]) : INT64_MAX;
         }
-        const unsigned mask = __reduce_or_sync(kFull, bit);
-        const unsigned upto = mask & (kFull >> (31 - lane));  // heads at lanes <= this one
-        const int hs = upto ? 31 - __clz(upto) : -1;          // this lane's segment head
-        const unsigned after = mask & ~(kFull >> (31 - lane)); // heads after this lane
-        const int se = after ? __ffs(after) - 2 : n - 1;      // last lane of this lane's segment
-        float2 v;
-        if (OP == kSoftmaxStats) {
-            const float s = lane < n ? x[c] : -INFINITY;
-            const float M = __shfl_sync(kFull, seg_scan<true>(s, lane, hs), se);
-            const float l = seg_scan<false>(lane < n ? expf(s - M) : 0.f, lane, hs);
-            v = make_float2(M, l);
-        } else {
-            v = make_float2(seg_scan<false>(lane < n ? x[c] : 0.f, lane, hs), 0.f);
-        }
-        const int nh = __popc(mask);
-        if (nh > 0) {
-            // the open row ends before the first head
-            const int h0 = __ffs(mask) - 1;
-            const float2 tail = shfl2(v, h0 > 0 ? h0 - 1 : 0);
-            const float2 total = h0 > 0 ? combine<OP>(acc, tail) : acc;
-            if (lane == 0) {
-                if (before) P.partial[2 * t] = total;
-                else P.out[P.nz_rows[cur]] = total;
-            }
-            // rows that start and end inside the chunk
-            const bool seg_end = lane < n - 1 && ((mask >> (lane + 1)) & 1u);
-            if (hs >= 0 && seg_end) P.out[P.nz_rows[cur + __popc(upto)]] = v;
-            // the last segment stays open
-            acc = shfl2(v, n - 1);
-            cur += nh;
-            before = false;
-        } else {
-            acc = combine<OP>(acc, shfl2(v, n - 1));
+        absorb<OP>(run, x[k]);
+    }
+
+    // segmented inclusive scan of the lanes' tails: a lane whose open segment
+    // starts inside it (at or after its first position) begins a segment
+    float2 v = run;  // identity for lanes without positions
+    bool f = starts_first || inner;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float2 pv = shfl2_up(v, o);
+        const bool pf = __shfl_up_sync(kFull, f, o);
+        if (lane >= o) {
+            if (!f) v = combine<OP>(pv, v);
+            f = f || pf;
         }
     }
-    if (lane == 0) {
-        if (before) P.partial[2 * t] = acc;
-        else if (P.nz_rowptr[cur + 1] > p0 + len) P.partial[2 * t + 1] = acc;
-        else P.out[P.nz_rows[cur]] = acc;
+    float2 excl = shfl2_up(v, 1);
+    if (lane == 0) excl = identity<OP>();
+    const bool next_starts = __shfl_down_sync(kFull, starts_first, 1);
+    const bool next_has = __shfl_down_sync(kFull, has_pos, 1);
+    auto write_row = [&](int64_t ri, float2 total, bool continues) {
+        if (ri == r0 && before) P.partial[2 * t] = total;        // row continued from the previous tile
+        else if (continues) P.partial[2 * t + 1] = total;        // row continued in the next tile
+        else P.out[P.nz_rows[ri]] = total;
+    };
+    // the row continued into this lane ends inside it
+    if (has_pos && !starts_first && inner) write_row(row_a0, combine<OP>(excl, head), false);
+    if (has_pos && lane < 31 && next_has) {
+        // the open row ends at this lane's last position
+        if (next_starts) write_row(row_i, v, false);
+    } else if (has_pos) {
+        // the last lane with positions: the row open at the tile's end
+        const int m = int(row_i - r0);
+        const int64_t end = m < nrs ? int64_t(rs[m]) : int64_t(P.nz_rowptr[row_i + 1]);
+        write_row(row_i, v, end > p0 + len);
     }
 }
 
