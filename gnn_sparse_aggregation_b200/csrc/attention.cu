@@ -9,17 +9,19 @@
 //
 // The scores come from the SDDMM walk of the forward CSR (owner Q[dst],
 // gathered K[src]) straight into the forward walk's window slots, where the
-// row statistics read them; they then go back to COO order once, for the
-// softmax.  The SpMMs run through this library's own entry points
-// (ag_spmm_fwd, ag_spmm_dx, and ag_backward for dV with dalpha in one walk);
-// the per-edge inputs of the backward's row reduction are first regrouped
-// into the forward walk's window-bucketed order; the row statistics m_r (maximum)
-// and l_r (sum of exp(s - m_r)) come from one segmented reduction over the
-// forward CSR, walked in the same edge-balanced tiles as the SpMM: one warp
-// per tile, each lane reducing its own run of consecutive positions in
-// registers, one Hillis-Steele segmented scan over the 32 lanes' open rows,
-// rows cut by a tile boundary finished by a fixup pass in tile order.  Every reduction tree
-// is fixed by the positions alone, so results are deterministic.
+// row statistics m_r (maximum) and l_r (sum of exp(s - m_r)) read them: one
+// segmented reduction over the forward CSR, walked in the same edge-balanced
+// tiles as the SpMM (one warp per tile, each lane reducing its own run of
+// consecutive positions in registers, one Hillis-Steele segmented scan over
+// the 32 lanes' open rows, rows cut by a tile boundary finished by a fixup
+// pass in tile order); the scores then go back to COO order once, for the
+// softmax pass, and the SpMMs run through this library's own entry points
+// (ag_spmm_fwd, ag_spmm_dx, and ag_backward for dV with dalpha in one walk).
+// Backward: c_r = sum over r's edges of alpha dalpha by the same segmented
+// reduction over copies regrouped into the forward walk's windows, then
+// ds_e = scale alpha_e (dalpha_e - c_dst) in one elementwise pass.  Every
+// reduction tree is fixed by the positions alone, so results are
+// deterministic.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -90,7 +92,10 @@ __device__ __forceinline__ void absorb(float2 &run, float s) {
 // (a_e alone when there is no b).
 template <int OP>
 __device__ __forceinline__ float leaf_value(const ReduceParams &P, int e) {
-    return OP == kSoftmaxStats ? P.scale * P.a[e] : (P.b ? P.a[e] * P.b[e] : P.a[e]);
+    // the rounded product (no contraction into a later subtraction): the
+    // softmax pass forms the same value, so exp(value - maximum) is exactly 1
+    // at the row's maximum
+    return OP == kSoftmaxStats ? __fmul_rn(P.scale, P.a[e]) : (P.b ? P.a[e] * P.b[e] : P.a[e]);
 }
 
 // One warp per tile of T consecutive forward-CSR positions.  Lane l owns the
@@ -105,6 +110,7 @@ __device__ __forceinline__ float leaf_value(const ReduceParams &P, int e) {
 // loaded before the reduction (the order map, then the values: two round
 // trips per tile).  Every combination order is fixed by the positions alone.
 constexpr int kMaxChunks = kMaxTileEdges / 32;  // positions per lane at most
+static_assert(kMaxChunks % 4 == 0, "16-byte loads of the order map");
 
 template <int OP>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const ReduceParams P) {
@@ -121,8 +127,19 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const Reduce
     const int a0 = lane * ppl;
     int e[kMaxChunks];
     float x[kMaxChunks];
+    if ((ppl & 3) == 0 && a0 + ppl <= len) {
+        // whole runs of a multiple of 4 positions: 16-byte loads (p0 and a0
+        // are multiples of 4 positions)
 #pragma unroll
-    for (int k = 0; k < kMaxChunks; ++k) e[k] = (k < ppl && a0 + k < len) ? __ldg(P.order + p0 + a0 + k) : -1;
+        for (int k = 0; k < kMaxChunks; k += 4) {
+            int4 v = make_int4(-1, -1, -1, -1);
+            if (k < ppl) v = __ldg(reinterpret_cast<const int4 *>(P.order + p0 + a0 + k));
+            e[k] = v.x, e[k + 1] = v.y, e[k + 2] = v.z, e[k + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < kMaxChunks; ++k) e[k] = (k < ppl && a0 + k < len) ? __ldg(P.order + p0 + a0 + k) : -1;
+    }
     const int64_t r0 = P.tile_nz[t];
     // rows r0 + 1 .. r_last: the row holding the next tile's first position
     // closes the range (the last tile: the last row)
@@ -218,7 +235,7 @@ __global__ void k_softmax_alpha(float *__restrict__ s, const int32_t *__restrict
                                 float scale, int64_t E) {
     for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
         const float2 r = ml[__ldcs(dst + e)];
-        s[e] = expf(scale * s[e] - r.x) / r.y;
+        s[e] = expf(__fmul_rn(scale, s[e]) - r.x) / r.y;
     }
 }
 

@@ -31,9 +31,20 @@ def agb():
     return lib()
 
 
-def _qkv(wl, dtype, seed=11):
+def _qkv(wl, dtype, seed=11, unaligned=False):
     mk = lambda s: workloads.features(wl.N, wl.H, dtype, seed * 1000 + s, DEV)
-    return mk(1), mk(2), mk(3), mk(4)   # Q, K, V, upstream gradient G
+    out = [mk(1), mk(2), mk(3), mk(4)]   # Q, K, V, upstream gradient G
+    if unaligned:
+        # the same values one element into a larger buffer: not 16-byte aligned
+        moved = []
+        for t in out:
+            big = torch.zeros(t.numel() + 1, dtype=dtype, device=DEV)
+            u = big[1:].view(t.shape)
+            u.copy_(t)
+            assert u.data_ptr() % 16 != 0
+            moved.append(u)
+        out = moved
+    return out
 
 
 def _row_rel(src, dst, N, Q, K, scale):
@@ -69,10 +80,10 @@ def _grad_bounds(src, dst, N, Q, K, V, G, scale, alpha, rel, tol):
     return bQ, bK, bV
 
 
-def _check_attention(agb, wl, dtype, what):
+def _check_attention(agb, wl, dtype, what, unaligned=False):
     import oracle
     g = agb.ag_graph_lower(wl.src, wl.dst, wl.N)
-    Q, K, V, G = _qkv(wl, dtype)
+    Q, K, V, G = _qkv(wl, dtype, unaligned=unaligned)
     scale = 1.0 / np.sqrt(wl.H)
     Y, alpha = agb.ag_attn_fwd(g, Q, K, V, scale)
     dQ, dK, dV = agb.ag_attn_backward(g, Q, K, V, scale, alpha, G)
@@ -119,6 +130,28 @@ def test_attention_narrow_and_ragged_widths(agb, H, dtype):
     dst = np.concatenate([rng.integers(0, N // 2, E), np.full(900, 5)])
     wl = workloads.custom(N, src, dst, H, seed=H, device=DEV)
     _check_attention(agb, wl, dtype, f"H={H}/{dtype}")
+
+
+@pytest.mark.parametrize("H,dtype", [(16, torch.float32), (32, torch.float32), (128, torch.float32),
+                                     (32, torch.bfloat16), (256, torch.bfloat16)])
+def test_attention_ring_widths(agb, H, dtype):
+    # every width whose rows are 4 to 32 16-byte vectors (the shared-memory
+    # ring walks), with one heavy row cut by tiles
+    rng = np.random.default_rng(100 + H)
+    N, E = 900, 9000
+    src = np.concatenate([rng.integers(0, N, E), rng.integers(0, N, 1500)])
+    dst = np.concatenate([rng.integers(0, 2 * N // 3, E), np.full(1500, 11)])
+    wl = workloads.custom(N, src, dst, H, seed=H, device=DEV)
+    _check_attention(agb, wl, dtype, f"ring H={H}/{dtype}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_attention_unaligned_inputs_take_the_register_walks(agb, dtype):
+    # unaligned Q, K, V and dY take the register walks of narrower vectors
+    # instead of the ring walks: the same bounds hold, and the results
+    # reproduce themselves
+    wl = workloads.make("sbm", seed=4, device=DEV)
+    _check_attention(agb, wl, dtype, f"unaligned/{dtype}", unaligned=True)
 
 
 def test_attention_skewed_rows_cut_by_many_tiles(agb):

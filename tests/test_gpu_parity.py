@@ -155,12 +155,11 @@ def test_unaligned_feature_pointers_take_the_narrow_path(agb, dtype):
     Y = g.fwd(wl.w, Xu)
     ref = g.fwd(wl.w, wl.X)
     torch.cuda.synchronize()
-    # The aligned input takes the paired walk, which sums the even and the odd
-    # positions of a row in the two halves of a warp and adds the two sums at
-    # the row end; the unaligned one takes a narrower walk that sums in
-    # position order.  Any summation order is acceptable within the tolerance
-    # (fp32 accumulation against the fp64 oracle), so both are checked there,
-    # and each must reproduce itself bit for bit.
+    # The aligned input takes the shared-memory ring walk of 16-byte vectors,
+    # the unaligned one a register walk of narrower vectors.  Any summation
+    # order is acceptable within the tolerance (fp32 accumulation against the
+    # fp64 oracle), so both are checked there, and each must reproduce itself
+    # bit for bit.
     import oracle
     want, bound = oracle.fwd(host(wl.src), host(wl.dst), N, host(wl.w), host(wl.X), with_bound=True)
     assert_within(Y, want, bound, TOL[dtype], "narrow path")
