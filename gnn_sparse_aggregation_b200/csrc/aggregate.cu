@@ -492,15 +492,27 @@ k_tiles_ring(const Params P) {
         la_end = P.nz_rowptr[la_base + gl + 1];
     }
     int la_k = 0;
+    // kRowScale: the open row's factor, and those of the look-ahead rows
+    // (fetched with the window, so that no row end waits on a load)
+    float row_inv = 0.f, la_inv = 0.f;
+    if constexpr ((MODE & kRowScale) != 0) {
+        if (active) row_inv = P.inv_cnt[row];
+        if (active && la_base + gl < P.n_nz) la_inv = P.inv_cnt[la_row];
+    }
 
     // indices: batch b (cur), b + 1 (nxt), b + 2 (nn); weights of b and b + 1
     int c_cur = 0, e_cur = 0, c_nxt = 0, e_nxt = 0, c_nn = 0, e_nn = 0;
     float w_cur = 0.f, w_nxt = 0.f;
+    // kEdgeScale: inv_cnt of the gathered column of this lane's position in
+    // batch b and b + 1 (loaded with the weights, used by weight and dot)
+    float sc_cur = 1.f, sc_nxt = 1.f;
     if (gl < len) { c_cur = __ldcs(P.col + p0 + gl); e_cur = __ldcs(P.order + p0 + gl); }
     if (G + gl < len) { c_nxt = __ldcs(P.col + p0 + G + gl); e_nxt = __ldcs(P.order + p0 + G + gl); }
+    if constexpr ((MODE & kEdgeScale) != 0)
+        if (gl < len) sc_cur = P.inv_cnt[c_cur];
     if ((MODE & kSpmm) && gl < len) {
         w_cur = load_w(P.w + e_cur);
-        if constexpr ((MODE & kEdgeScale) != 0) w_cur *= P.inv_cnt[c_cur];
+        if constexpr ((MODE & kEdgeScale) != 0) w_cur *= sc_cur;
     }
 
     const uint32_t row_bytes = uint32_t(H) * sizeof(T);
@@ -543,7 +555,7 @@ k_tiles_ring(const Params P) {
             store_slot<VEC, NV>(slot, 0, G, colok, o);
         } else {
             if constexpr ((MODE & kRowScale) != 0) {
-                const float r = P.inv_cnt[row];
+                const float r = row_inv;
 #pragma unroll
                 for (int k = 0; k < NV; ++k)
 #pragma unroll
@@ -562,6 +574,7 @@ k_tiles_ring(const Params P) {
         before = false;
         row = __shfl_sync(gmask, la_row, la_k, G);
         rend = __shfl_sync(gmask, la_end, la_k, G);
+        if constexpr ((MODE & kRowScale) != 0) row_inv = __shfl_sync(gmask, la_inv, la_k, G);
         if (++la_k == G) {
             la_base += G;
             la_k = 0;
@@ -570,6 +583,7 @@ k_tiles_ring(const Params P) {
             if (la_base + gl < P.n_nz) {
                 la_row = P.nz_rows[la_base + gl];
                 la_end = P.nz_rowptr[la_base + gl + 1];
+                if constexpr ((MODE & kRowScale) != 0) la_inv = P.inv_cnt[la_row];
             }
         }
         if ((MODE & kSddmm)) {
@@ -623,13 +637,15 @@ k_tiles_ring(const Params P) {
 
     for (int base = 0; base < len_max; base += G) {
         if (base > 0) {
-            c_cur = c_nxt; e_cur = e_nxt; w_cur = w_nxt;
+            c_cur = c_nxt; e_cur = e_nxt; w_cur = w_nxt; sc_cur = sc_nxt;
             c_nxt = c_nn; e_nxt = e_nn;
         }
         // weights of the next batch, indices of the one after
         if ((MODE & kSpmm)) w_nxt = (base + G + gl < len) ? load_w(P.w + e_nxt) : 0.f;
-        if constexpr ((MODE & kEdgeScale) != 0)
-            if (base + G + gl < len) w_nxt *= P.inv_cnt[c_nxt];
+        if constexpr ((MODE & kEdgeScale) != 0) {
+            sc_nxt = (base + G + gl < len) ? P.inv_cnt[c_nxt] : 1.f;
+            w_nxt *= sc_nxt;
+        }
         c_nn = 0;
         e_nn = 0;
         if (base + 2 * G + gl < len) {
@@ -657,7 +673,7 @@ k_tiles_ring(const Params P) {
                 if ((MODE & kSddmm)) {
                     const float d = reduce_chunk<U, G>(dots, gl, FULL);
                     if ((gl & ~(U - 1)) == j0)  // lane j0 + t: position j0 + t
-                        P.dw[e_cur] = (MODE & kEdgeScale) ? d * P.inv_cnt[c_cur] : d;
+                        P.dw[e_cur] = (MODE & kEdgeScale) ? d * sc_cur : d;
                 }
             }
         } else {
@@ -668,7 +684,7 @@ k_tiles_ring(const Params P) {
                 if ((MODE & kSddmm)) {
 #pragma unroll
                     for (int o = G / 2; o > 0; o >>= 1) d += __shfl_xor_sync(FULL, d, o, G);
-                    if (gl == j && base + j < len) P.dw[e_cur] = (MODE & kEdgeScale) ? d * P.inv_cnt[c_cur] : d;
+                    if (gl == j && base + j < len) P.dw[e_cur] = (MODE & kEdgeScale) ? d * sc_cur : d;
                 }
                 refill(base, j, j % D, j + D < G ? c_cur : c_nxt, true);
             }
