@@ -1720,13 +1720,36 @@ __global__ void k_zero2(float2 *__restrict__ p, int64_t n) {
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
         p[i] = make_float2(0.f, 0.f);
 }
-// out[e] = dis[src_e] * w_e * dis[dst_e] in COO order (w = null: 1)
+// out[e] = dis[src_e] * w_e * dis[dst_e] in COO order (w = null: 1).  Each
+// thread keeps kGcnUnroll edges in flight (strided by the grid, so the
+// warp's loads stay coalesced): all endpoint and weight loads, then all
+// gathers from the L2-resident dis, then the products.
+constexpr int kGcnUnroll = 4;
 __global__ void k_gcn_weights(const int32_t *__restrict__ src, const int32_t *__restrict__ dst,
                               const float *__restrict__ w, const float *__restrict__ dis, int64_t E,
                               float *__restrict__ out) {
-    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
-        const float we = w ? __ldcs(w + e) : 1.f;
-        __stcs(out + e, dis[__ldcs(src + e)] * we * dis[__ldcs(dst + e)]);
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t e0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e0 < E; e0 += stride * kGcnUnroll) {
+        int a[kGcnUnroll], b[kGcnUnroll];
+        float we[kGcnUnroll], da[kGcnUnroll], db[kGcnUnroll];
+#pragma unroll
+        for (int k = 0; k < kGcnUnroll; ++k) {
+            const int64_t e = e0 + k * stride;
+            a[k] = e < E ? __ldcs(src + e) : 0;
+            b[k] = e < E ? __ldcs(dst + e) : 0;
+            we[k] = (w && e < E) ? __ldcs(w + e) : 1.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kGcnUnroll; ++k) {
+            const bool ok = e0 + k * stride < E;
+            da[k] = ok ? dis[a[k]] : 0.f;
+            db[k] = ok ? dis[b[k]] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kGcnUnroll; ++k) {
+            const int64_t e = e0 + k * stride;
+            if (e < E) __stcs(out + e, da[k] * we[k] * db[k]);
+        }
     }
 }
 unsigned flat_grid(int64_t n) {

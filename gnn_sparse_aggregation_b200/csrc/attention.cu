@@ -218,11 +218,29 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const Reduce
 }
 
 // Rows cut by tile boundaries: out[row] = slot(2 first + 1) combined with
-// slot(2 t) for t = first + 1 .. last, in tile order (one thread per row).
+// the slots 2t of tiles t = first + 1 .. last.  The n_long long spans (listed
+// first) take one warp each: lane l combines the tiles first + 1 + l + 32 i
+// in order, then a butterfly of fixed shape combines the lanes, so no thread
+// waits on a chain of hundreds of loads; every other span takes one thread
+// and combines in tile order.
 template <int OP>
-__global__ void k_row_reduce_fixup(const int4 *__restrict__ spans, int64_t n_span, const float2 *__restrict__ partial,
-                                   float2 *__restrict__ out) {
-    const int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+__global__ void k_row_reduce_fixup(const int4 *__restrict__ spans, int64_t n_span, int64_t n_long,
+                                   const float2 *__restrict__ partial, float2 *__restrict__ out) {
+    const int64_t gt = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gt < n_long * 32) {  // whole warps (n_long * 32 is a multiple of 32)
+        const int lane = threadIdx.x & 31;
+        const int4 sp = spans[gt >> 5];
+        float2 v = identity<OP>();
+        for (int64_t t = int64_t(sp.y) + 1 + lane; t <= sp.z; t += 32) v = combine<OP>(v, partial[2 * t]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float2 u = make_float2(__shfl_xor_sync(kFull, v.x, o), __shfl_xor_sync(kFull, v.y, o));
+            v = (lane & o) ? combine<OP>(u, v) : combine<OP>(v, u);
+        }
+        if (lane == 0) out[sp.x] = combine<OP>(partial[2 * int64_t(sp.y) + 1], v);
+        return;
+    }
+    const int64_t s = n_long + (gt - n_long * 32);
     if (s >= n_span) return;
     const int4 sp = spans[s];
     float2 v = partial[2 * int64_t(sp.y) + 1];
@@ -230,20 +248,58 @@ __global__ void k_row_reduce_fixup(const int4 *__restrict__ spans, int64_t n_spa
     out[sp.x] = v;
 }
 
+// The two per-edge passes below gather one per-row value per edge from an
+// L2-resident table: each thread keeps kEdgeUnroll edges in flight (strided
+// by the grid, so every load of the warp stays coalesced), loading all
+// their inputs before the gathers and all gathers before the arithmetic.
+constexpr int kEdgeUnroll = 4;
+
 // alpha_e = exp(scale * s_e - m_r) / l_r (in place over s)
 __global__ void k_softmax_alpha(float *__restrict__ s, const int32_t *__restrict__ dst, const float2 *__restrict__ ml,
                                 float scale, int64_t E) {
-    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
-        const float2 r = ml[__ldcs(dst + e)];
-        s[e] = expf(__fmul_rn(scale, s[e]) - r.x) / r.y;
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t e0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e0 < E; e0 += stride * kEdgeUnroll) {
+        int d[kEdgeUnroll];
+        float v[kEdgeUnroll];
+        float2 r[kEdgeUnroll];
+#pragma unroll
+        for (int k = 0; k < kEdgeUnroll; ++k) {
+            const int64_t e = e0 + k * stride;
+            d[k] = e < E ? __ldcs(dst + e) : 0;
+            v[k] = e < E ? s[e] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kEdgeUnroll; ++k) r[k] = e0 + k * stride < E ? ml[d[k]] : make_float2(0.f, 1.f);
+#pragma unroll
+        for (int k = 0; k < kEdgeUnroll; ++k) {
+            const int64_t e = e0 + k * stride;
+            if (e < E) s[e] = expf(__fmul_rn(scale, v[k]) - r[k].x) / r[k].y;
+        }
     }
 }
 
 // ds_e = scale * alpha_e * (dalpha_e - c_r) (in place over dalpha)
 __global__ void k_attn_ds(const float *__restrict__ alpha, float *__restrict__ da, const int32_t *__restrict__ dst,
                           const float2 *__restrict__ c, float scale, int64_t E) {
-    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x)
-        da[e] = scale * alpha[e] * (da[e] - c[__ldcs(dst + e)].x);
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t e0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e0 < E; e0 += stride * kEdgeUnroll) {
+        int d[kEdgeUnroll];
+        float a[kEdgeUnroll], g[kEdgeUnroll], cr[kEdgeUnroll];
+#pragma unroll
+        for (int k = 0; k < kEdgeUnroll; ++k) {
+            const int64_t e = e0 + k * stride;
+            d[k] = e < E ? __ldcs(dst + e) : 0;
+            a[k] = e < E ? __ldcs(alpha + e) : 0.f;
+            g[k] = e < E ? da[e] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kEdgeUnroll; ++k) cr[k] = e0 + k * stride < E ? c[d[k]].x : 0.f;
+#pragma unroll
+        for (int k = 0; k < kEdgeUnroll; ++k) {
+            const int64_t e = e0 + k * stride;
+            if (e < E) da[e] = scale * a[k] * (g[k] - cr[k]);
+        }
+    }
 }
 
 unsigned flat_blocks(int64_t n) {
@@ -290,8 +346,11 @@ int row_reduce(const ag_graph *g, const float *a_b, const float *b_b, float scal
         const unsigned grid = unsigned((g->n_tiles + kWarpsPerBlock - 1) / kWarpsPerBlock);
         k_row_reduce<OP><<<grid, kWarpsPerBlock * 32, 0, st>>>(P);
     }
-    if (D.n_span > 0)
-        k_row_reduce_fixup<OP><<<unsigned((D.n_span + 255) / 256), 256, 0, st>>>(D.spans, D.n_span, partial, out);
+    if (D.n_span > 0) {
+        const int64_t threads = D.n_span_long * 32 + (D.n_span - D.n_span_long);
+        k_row_reduce_fixup<OP><<<unsigned((threads + 255) / 256), 256, 0, st>>>(D.spans, D.n_span, D.n_span_long,
+                                                                                partial, out);
+    }
     cudaError_t err = cudaGetLastError();
     return err == cudaSuccess ? AG_OK : cuda_fail(err, "row reduction");
 }
