@@ -1367,6 +1367,7 @@ size_t scratch_needed(const ag_graph *g, int64_t H) {
 struct EdgeScale {
     const int32_t *dst = nullptr;     // COO destinations [E]
     const int32_t *rowptr = nullptr;  // forward CSR row pointers [N + 1]
+    const float *mul = nullptr;       // into buckets only: multiply edge e's value by mul[e] first
 };
 __device__ __forceinline__ float per_dst(float v, const EdgeScale &sc, int64_t e) {
     const int d = __ldcs(sc.dst + e);
@@ -1382,6 +1383,7 @@ __global__ void k_bucket_scatter(const float *__restrict__ w, const int32_t *__r
                                  EdgeScale sc, float *__restrict__ w_b) {
     for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < E; e += int64_t(gridDim.x) * blockDim.x) {
         float v = w ? __ldcs(w + e) : 1.f;
+        if (sc.mul) v *= __ldcs(sc.mul + e);
         if (SCALED) v = per_dst(v, sc, e);
         w_b[__ldcs(slot + e)] = v;
     }
@@ -1425,6 +1427,13 @@ k_bucket_staged(const float *__restrict__ in, const int32_t *__restrict__ slot,
         const int i = k * kThreads + threadIdx.x;
         sl[k] = i < n ? __ldcs(slot + c0 + i) : -1;
         v[k] = (TO_BUCKETS && i < n) ? (in ? __ldcs(in + c0 + i) : 1.f) : 0.f;
+    }
+    if (TO_BUCKETS && sc.mul) {
+#pragma unroll
+        for (int k = 0; k < kStageItems; ++k) {
+            const int i = k * kThreads + threadIdx.x;
+            if (i < n) v[k] *= __ldcs(sc.mul + c0 + i);
+        }
     }
     if constexpr (SCALED) {
         // destinations of all items, then their row lengths: two waves of
@@ -1842,6 +1851,12 @@ size_t spmm_scratch_edge_offset(const ag_graph *g, int64_t H, int which) {
 }
 void regroup_to_buckets(const ag_graph *g, int d, const float *in, float *out_b, cudaStream_t st) {
     regroup(true, g->dir[d], in, g->E, out_b, st);
+}
+void regroup_product_to_buckets(const ag_graph *g, int d, const float *a, const float *b, float *out_b,
+                                cudaStream_t st) {
+    EdgeScale sc;
+    sc.mul = b;
+    regroup(true, g->dir[d], a, g->E, out_b, st, sc);
 }
 
 }  // namespace ag

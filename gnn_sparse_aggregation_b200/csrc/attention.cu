@@ -18,7 +18,7 @@
 // softmax pass, and the SpMMs run through this library's own entry points
 // (ag_spmm_fwd, ag_spmm_dx, and ag_backward for dV with dalpha in one walk).
 // Backward: c_r = sum over r's edges of alpha dalpha by the same segmented
-// reduction over copies regrouped into the forward walk's windows, then
+// reduction over the products, regrouped into the forward walk's windows, then
 // ds_e = scale alpha_e (dalpha_e - c_dst) in one elementwise pass.  Every
 // reduction tree is fixed by the positions alone, so results are
 // deterministic.
@@ -444,14 +444,13 @@ int ag_attn_backward(const ag_graph *g, const void *Q, const void *K, const void
         // dV = A_alpha^T dY and dalpha_e = dot(V[src], dY[dst]) in one transpose
         // walk (the weighted-sum backward with weights alpha and "features" V)
         if ((rc = ag_backward(g, alpha, V, dY, dV, ds, H, dtype, sp, spmm_bytes, stream)) != AG_OK) return rc;
-        // c_r = sum over r's edges of alpha dalpha, from bucket-ordered copies
-        // (the SpMM scratch's two per-edge arrays are free between the walks)
+        // c_r = sum over r's edges of alpha dalpha: the products, formed while
+        // regrouping into the forward windows (the SpMM scratch's per-edge
+        // arrays are free between the walks), summed per row
         float2 *c = reinterpret_cast<float2 *>(scr + L.rows);
-        float *a_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 0));
-        float *d_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 1));
-        regroup_to_buckets(g, 0, alpha, a_b, st);
-        regroup_to_buckets(g, 0, ds, d_b, st);
-        rc = row_reduce<kSum>(g, a_b, d_b, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
+        float *p_b = reinterpret_cast<float *>(scr + L.spmm + spmm_scratch_edge_offset(g, H, 0));
+        regroup_product_to_buckets(g, 0, alpha, ds, p_b, st);
+        rc = row_reduce<kSum>(g, p_b, nullptr, 1.f, reinterpret_cast<float2 *>(scr + L.partial), c, st);
         if (rc != AG_OK) return rc;
         k_attn_ds<<<flat_blocks(g->E), 256, 0, st>>>(alpha, ds, g->coo_dst, c, scale, g->E);
         cudaError_t err = cudaGetLastError();

@@ -108,6 +108,9 @@ size_t spmm_scratch_edge_offset(const ag_graph *g, int64_t H, int which);
 // out_b[bucket slot of COO edge e] = in[e] for the walk direction d: COO
 // order into the window-bucketed order the walks read through bucket_of_pos.
 void regroup_to_buckets(const ag_graph *g, int d, const float *in, float *out_b, cudaStream_t st);
+// out_b[bucket slot of COO edge e] = a[e] * b[e] for the walk direction d.
+void regroup_product_to_buckets(const ag_graph *g, int d, const float *a, const float *b, float *out_b,
+                                cudaStream_t st);
 // out[e] = in_b[bucket slot of COO edge e]: back to COO order.
 void regroup_from_buckets(const ag_graph *g, int d, const float *in_b, float *out, cudaStream_t st);
 // out[r].x = sum of a_b over the forward-CSR positions of every row r with
