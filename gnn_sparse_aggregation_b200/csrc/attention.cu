@@ -110,6 +110,7 @@ __device__ __forceinline__ float leaf_value(const ReduceParams &P, int e) {
 // loaded before the reduction (the order map, then the values: two round
 // trips per tile).  Every combination order is fixed by the positions alone.
 constexpr int kMaxChunks = kMaxTileEdges / 32;  // positions per lane at most
+constexpr int kStageUnroll = 8;                  // row starts in flight per lane while staging
 static_assert(kMaxChunks % 4 == 0, "16-byte loads of the order map");
 
 template <int OP>
@@ -145,11 +146,26 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_row_reduce(const Reduce
     // closes the range (the last tile: the last row)
     const int64_t r_last = t + 1 < P.n_tiles ? P.tile_nz[t + 1] : P.n_nz - 1;
     const int nrs = int(r_last - r0);  // <= T: at most one row starts per position
-    for (int i = lane; i < nrs; i += 32) rs[i] = P.nz_rowptr[r0 + 1 + i];
     const int64_t first_start = P.nz_rowptr[r0];  // start of the tile's first row
-    const bool before = first_start < p0;
+    // the leaves (their gathers in flight while the row starts are staged)
 #pragma unroll
     for (int k = 0; k < kMaxChunks; ++k) x[k] = e[k] >= 0 ? leaf_value<OP>(P, e[k]) : 0.f;
+    // kStageUnroll loads in flight per lane before their stores (a tile of
+    // short rows stages up to T starts: one round trip per 8 x 32 of them)
+    for (int i0 = 0; i0 < nrs; i0 += 32 * kStageUnroll) {
+        int v[kStageUnroll];
+#pragma unroll
+        for (int u = 0; u < kStageUnroll; ++u) {
+            const int i = i0 + 32 * u + lane;
+            v[u] = i < nrs ? __ldg(P.nz_rowptr + r0 + 1 + i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kStageUnroll; ++u) {
+            const int i = i0 + 32 * u + lane;
+            if (i < nrs) rs[i] = v[u];
+        }
+    }
+    const bool before = first_start < p0;
     __syncwarp();
 
     // the row holding this lane's first position: r0 + the number of staged
