@@ -364,7 +364,10 @@ AG_API int ag_step_host(const ag_graph *g, const float *w_host, const void *X_ho
  * step's fused backward pass on the same staging buffer, not after that
  * step's copies out.  Back-to-back steps on one staging buffer therefore
  * bring the next step's inputs in while the previous step's dX and dw go out.
- * `stream` is still ordered after every copy of this call.
+ * `stream` is still ordered after every copy of this call.  Steps that
+ * alternate between two staging buffers, each with its own `stream` (and
+ * its own host outputs), overlap further: a step's copies in wait only for
+ * the backward pass two steps back, and its compute only for its inputs.
  *
  * The staging buffer belongs to the steps between calls: no other work may
  * read or write it.  The first call on a buffer (or on one of more than 16

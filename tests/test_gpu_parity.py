@@ -374,6 +374,37 @@ def test_pipelined_steps_keep_each_steps_results(agb, modes):
         assert torch.equal(hdw, dw), k
 
 
+def test_pipelined_steps_on_two_staging_buffers_and_two_streams(agb):
+    """The bench's end-to-end pattern: pipelined steps alternating between two
+    staging buffers, each on its own stream, so that a step's copies in and
+    compute can overlap the previous step's compute and copies out.  Every
+    step must return exactly its own results (different inputs per step)."""
+    src, dst = workloads.rmat_edges(17, 16, seed=8)
+    N = 1 << 17
+    wl, g = graph(agb, N, src.numpy(), dst.numpy(), 64, torch.bfloat16)
+    nbytes = agb.ag_step_staging_bytes(g, wl.H, torch.bfloat16)
+    stagings = [torch.empty(nbytes, dtype=torch.uint8, device=DEV) for _ in range(2)]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    ins, outs, refs = [], [], []
+    for k in range(6):
+        w = wl.w * (k + 1)
+        X = (wl.X.float() * (k + 1) - k).bfloat16()
+        dY = (wl.dY.float() + k).bfloat16()
+        refs.append(tuple(t.cpu() for t in (g.fwd(w, X), *g.backward(w, X, dY))))
+        ins.append(tuple(t.cpu().pin_memory() for t in (w, X, dY)))
+        outs.append((torch.empty_like(ins[-1][1]).pin_memory(), torch.empty_like(ins[-1][1]).pin_memory(),
+                     torch.empty_like(ins[-1][0]).pin_memory()))
+    torch.cuda.synchronize()
+    for k, ((hw, hX, hdY), (hY, hdX, hdw)) in enumerate(zip(ins, outs)):
+        agb.ag_step_host_pipelined(g, hw, hX, hdY, hY, hdX, hdw, stagings[k % 2], stream=streams[k % 2])
+    for st in streams:
+        st.synchronize()
+    for k, ((hY, hdX, hdw), (Y, dX, dw)) in enumerate(zip(outs, refs)):
+        assert torch.equal(hY.view(torch.int16), Y.view(torch.int16)), k
+        assert torch.equal(hdX.view(torch.int16), dX.view(torch.int16)), k
+        assert torch.equal(hdw, dw), k
+
+
 def test_pipelined_steps_with_a_new_layout_on_the_same_buffer(agb):
     """Pipelined steps of different widths (and dtypes) back to back on one
     staging buffer: a step whose layout differs from the previous step's must
