@@ -165,19 +165,33 @@ def traffic_key(args):
     return args.workload if args.rmat_scale is None else f"{args.workload}@scale{args.rmat_scale}"
 
 
-def ncu_traffic(workload, kernel_op):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken on
-    the current kernel sources (else None)."""
+def ncu_record(workload, kernel_op):
+    """The committed ncu record of one entry point, if it was taken on the
+    current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         rec = d.get(workload, {}).get(kernel_op)
         if rec and rec.get("source_hash") == source_hash():
-            return rec.get("bytes_per_launch")
+            return rec
     except Exception:
         pass
     return None
+
+
+def ncu_traffic(workload, kernel_op):
+    """DRAM bytes per launch from a committed ncu capture (else None)."""
+    rec = ncu_record(workload, kernel_op)
+    return rec.get("bytes_per_launch") if rec else None
+
+
+def ncu_l2_hit(workload, kernel_op):
+    """L2 sector hit rate of the entry point's walk from the committed
+    small-case capture (R-MAT scale 20: the counter takes several passes),
+    with the kernel and the case it was taken on (else None)."""
+    rec = ncu_record(workload, kernel_op)
+    return rec.get("l2_hit") if rec else None
 
 
 class ClockSampler:
@@ -543,6 +557,9 @@ def our_arm(args):
         if dram:  # measured DRAM bytes of the call (ncu) over its live time: the DRAM fraction
             kernels[op]["dram_bytes"] = dram
             kernels[op]["dram_frac_of_peak"] = dram_frac(dram, avg[op], hbm)
+        hit = ncu_l2_hit(traffic_key(args), op)
+        if hit:
+            kernels[op]["l2_hit"] = hit
     traffic = ncu_traffic(traffic_key(args), dominant)
     launches_per_step = launches_per_step_of(st, wl)
     line = {
@@ -559,7 +576,8 @@ def our_arm(args):
                      "frac": algo[dominant] / (avg[dominant] / 1e3) / 1e9 / hbm,
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "traffic": traffic,
-                     "dram_frac": dram_frac(traffic, avg[dominant], hbm) if traffic else None},
+                     "dram_frac": dram_frac(traffic, avg[dominant], hbm) if traffic else None,
+                     "l2_hit": ncu_l2_hit(traffic_key(args), dominant)},
         "kernels": kernels,
         "lowering_ms": lower_ms[1], "lowering_first_call_ms": lower_ms[0],
         "schedule": {k: st[k] for k in ("tile_edges", "tiles", "spanning_rows_f", "long_spanning_rows_f",
