@@ -103,12 +103,13 @@ __device__ __forceinline__ float leaf_value(const ReduceParams &P, int e) {
 // them in order in registers: every row that starts and ends inside the lane
 // is finished there; the lane's head (the positions before its first row
 // start) and its tail (the row open at its end) are combined across lanes
-// with one segmented scan over the 32 tails.  The tile's row starts are
-// staged in shared memory first; a lane finds its first row by a binary
-// search there.  kSoftmaxStats keeps (max, sum of exp(s - max)) per segment,
-// rescaling the sum when the maximum grows; kSum keeps a sum.  All leaves are
-// loaded before the reduction (the order map, then the values: two round
-// trips per tile).  Every combination order is fixed by the positions alone.
+// with one segmented scan over the 32 tails.  All leaves are loaded before
+// the reduction (the order map, then the values: two round trips per tile);
+// while the values are in flight the tile's row starts are staged in shared
+// memory, where a lane finds its first row by a binary search.
+// kSoftmaxStats keeps (max, sum of exp(s - max)) per segment, rescaling the
+// sum when the maximum grows; kSum keeps a sum.  Every combination order is
+// fixed by the positions alone.
 constexpr int kMaxChunks = kMaxTileEdges / 32;  // positions per lane at most
 constexpr int kStageUnroll = 8;                  // row starts in flight per lane while staging
 static_assert(kMaxChunks % 4 == 0, "16-byte loads of the order map");
