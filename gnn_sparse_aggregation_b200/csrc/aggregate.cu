@@ -61,6 +61,14 @@ namespace {
 #endif
 
 constexpr int kThreads = 256;
+// Blocks of the ring walk: tiles vary in length, and a smaller block frees
+// its share of an SM as soon as its few slowest groups finish (at R-MAT-22
+// the step took 2 % less time with 128 threads than with 256; 512 was
+// slower); occupancy per SM is the same.
+#ifndef AG_RING_THREADS
+#define AG_RING_THREADS 128
+#endif
+constexpr int kRingThreads = AG_RING_THREADS;
 constexpr int kUnroll = 4;     // gathered rows in flight per lane (register path)
 constexpr int kMinBlocks = 4;  // resident CTAs per SM the register path is compiled for
 constexpr int kRingDepth = AG_RING_DEPTH;
@@ -427,7 +435,7 @@ template <typename T, int NV, int VEC> struct RowAcc {
 // gathered dY row feeds the feature-gradient row of its source and the dot
 // product of its edge.  Rows are accumulated with scalar fp32 FMAs.
 template <typename T, int VEC, int NV, int G, int MODE, int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kRingThreads)
 k_tiles_ring(const Params P) {
     using raw_t = typename Vec<T, VEC>::raw;
     static_assert(sizeof(raw_t) == 16, "ring path moves 16-byte vectors");
@@ -435,7 +443,7 @@ k_tiles_ring(const Params P) {
     constexpr unsigned FULL = 0xffffffffu;
     extern __shared__ uint4 ring[];
     constexpr int LOG2G = G == 32 ? 5 : G == 16 ? 4 : G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
-    const int64_t gid = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> LOG2G;
+    const int64_t gid = (int64_t(blockIdx.x) * kRingThreads + threadIdx.x) >> LOG2G;
     const int64_t n_tiles_pad = (P.n_tiles + (32 / G) - 1) / (32 / G) * (32 / G);
     const int gl = threadIdx.x & (G - 1);
     const int lane = threadIdx.x & 31;
@@ -1193,9 +1201,9 @@ void launch_ring(const Params &P, cudaStream_t st) {
     // tile groups padded to whole warps, then the empty-row groups
     const int64_t per_warp = 32 / G;
     const int64_t groups = (P.n_tiles + per_warp - 1) / per_warp * per_warp + P.n_zero;
-    const unsigned grid = unsigned((groups + kThreads / G - 1) / (kThreads / G));
+    const unsigned grid = unsigned((groups + kRingThreads / G - 1) / (kRingThreads / G));
     // ring: D slots x NV vectors x 16 bytes for every lane of the block
-    const size_t smem = size_t(kThreads) * D * NV * 16;
+    const size_t smem = size_t(kRingThreads) * D * NV * 16;
     // the shared-memory limit is an attribute of the function in each device's
     // context: set it once per device (a race only repeats the same call)
     static std::atomic<uint64_t> configured{0};
@@ -1207,7 +1215,7 @@ void launch_ring(const Params &P, cudaStream_t st) {
                              int(smem));
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    k_tiles_ring<T, VEC, NV, G, MODE, D><<<grid, kThreads, smem, st>>>(P);
+    k_tiles_ring<T, VEC, NV, G, MODE, D><<<grid, kRingThreads, smem, st>>>(P);
 }
 
 template <typename T, int VEC, int NV, int MODE>
