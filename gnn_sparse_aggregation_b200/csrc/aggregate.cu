@@ -69,6 +69,10 @@ constexpr int kThreads = 256;
 #define AG_RING_THREADS 128
 #endif
 constexpr int kRingThreads = AG_RING_THREADS;
+#ifndef AG_WALK_THREADS
+#define AG_WALK_THREADS 256  // blocks of the one-warp-per-tile walk (1 KB rows)
+#endif
+constexpr int kWalkThreads = AG_WALK_THREADS;
 constexpr int kUnroll = 4;     // gathered rows in flight per lane (register path)
 constexpr int kMinBlocks = 4;  // resident CTAs per SM the register path is compiled for
 constexpr int kRingDepth = AG_RING_DEPTH;
@@ -833,10 +837,12 @@ __device__ __forceinline__ void load_rows(const Params &P, int64_t base, int lan
 }
 
 // resident CTAs per SM the walk is compiled for (a register budget)
-constexpr int walk_min_blocks(int MODE) { return (MODE & kSddmm) ? 2 : 4; }
+// resident blocks the warp walk is compiled for: 1024 (SpMM) or 512 (with
+// the dot product) threads per SM, whatever the block size
+constexpr int walk_min_blocks(int MODE) { return ((MODE & kSddmm) ? 512 : 1024) / kWalkThreads; }
 
 template <typename T, int LB, int MODE>
-__global__ void __launch_bounds__(kThreads, walk_min_blocks(MODE)) k_walk(const Params P) {
+__global__ void __launch_bounds__(kWalkThreads, walk_min_blocks(MODE)) k_walk(const Params P) {
     using S = Slice<LB>;
     constexpr unsigned FULL = 0xffffffffu;
     constexpr int VPL = LB / int(sizeof(T));
@@ -846,11 +852,11 @@ __global__ void __launch_bounds__(kThreads, walk_min_blocks(MODE)) k_walk(const 
     static_assert(32 % D == 0 && (D >= CH ? D % CH == 0 : CH % D == 0), "chunk shapes");
     constexpr bool SPMM = (MODE & kSpmm) != 0, SDDMM = (MODE & kSddmm) != 0;
     constexpr bool ROW_SCALE = (MODE & kRowScale) != 0, EDGE_SCALE = (MODE & kEdgeScale) != 0;
-    extern __shared__ uint4 walk_ring[];  // (kThreads / 32) * kWalkRingBytes bytes
+    extern __shared__ uint4 walk_ring[];  // (kWalkThreads / 32) * kWalkRingBytes bytes
     char *ring = reinterpret_cast<char *>(walk_ring);
 
     const int lane = threadIdx.x & 31;
-    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t warp = (int64_t(blockIdx.x) * kWalkThreads + threadIdx.x) >> 5;
     const int lane_off = lane * S::SEGB;
     if (warp >= P.n_tiles) {  // trailing warps: rows without edges get zeros
         const int64_t z0 = (warp - P.n_tiles) * kZeroRowsPerWarp;
@@ -1261,8 +1267,8 @@ void dispatch_nv(const Params &P, const Shape &s, cudaStream_t st) {
 template <typename T, int LB, int MODE>
 void launch_walk(const Params &P, cudaStream_t st) {
     const int64_t warps = P.n_tiles + (P.n_zero + kZeroRowsPerWarp - 1) / kZeroRowsPerWarp;
-    const unsigned grid = unsigned((warps + kThreads / 32 - 1) / (kThreads / 32));
-    const size_t smem = size_t(kThreads / 32) * kWalkRingBytes;
+    const unsigned grid = unsigned((warps + kWalkThreads / 32 - 1) / (kWalkThreads / 32));
+    const size_t smem = size_t(kWalkThreads / 32) * kWalkRingBytes;
     // the shared-memory limit is an attribute of the function in each device's
     // context: set it once per device (a race only repeats the same call)
     static std::atomic<uint64_t> configured{0};
@@ -1273,7 +1279,7 @@ void launch_walk(const Params &P, cudaStream_t st) {
         cudaFuncSetAttribute(k_walk<T, LB, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    if (grid > 0) k_walk<T, LB, MODE><<<grid, kThreads, smem, st>>>(P);
+    if (grid > 0) k_walk<T, LB, MODE><<<grid, kWalkThreads, smem, st>>>(P);
 }
 
 template <int MODE, typename T>
