@@ -63,8 +63,10 @@ namespace {
 constexpr int kThreads = 256;
 // Blocks of the ring walk: tiles vary in length, and a smaller block frees
 // its share of an SM as soon as its few slowest groups finish (at R-MAT-22
-// the step took 2 % less time with 128 threads than with 256; 512 was
-// slower); occupancy per SM is the same.
+// the step took 4 % less time with 128 threads than with 256, the fused
+// backward walk 5 % less; 64 and 512 were slower); occupancy per SM is the
+// same.  The row-scaled forward walk of the mean measured 0.3 ms slower with
+// 128 threads and keeps 256.
 #ifndef AG_RING_THREADS
 #define AG_RING_THREADS 128
 #endif
@@ -83,6 +85,7 @@ constexpr int kChunk = AG_CHUNK;
 // (forward mean); kEdgeScale multiplies every edge's weight and dot product
 // by inv_cnt of its gathered column (the destination, in the transpose walk).
 enum Mode { kSpmm = 1, kSddmm = 2, kBoth = 3, kRowScale = 4, kEdgeScale = 8 };
+constexpr int ring_threads(int MODE) { return (MODE & kRowScale) ? 256 : kRingThreads; }
 
 // A weight looked up through the bucketed layout: each 128-byte line of a
 // window is used by about 32 positions of that window's tiles, so it is kept
@@ -439,7 +442,7 @@ template <typename T, int NV, int VEC> struct RowAcc {
 // gathered dY row feeds the feature-gradient row of its source and the dot
 // product of its edge.  Rows are accumulated with scalar fp32 FMAs.
 template <typename T, int VEC, int NV, int G, int MODE, int D>
-__global__ void __launch_bounds__(kRingThreads)
+__global__ void __launch_bounds__(ring_threads(MODE))
 k_tiles_ring(const Params P) {
     using raw_t = typename Vec<T, VEC>::raw;
     static_assert(sizeof(raw_t) == 16, "ring path moves 16-byte vectors");
@@ -447,7 +450,7 @@ k_tiles_ring(const Params P) {
     constexpr unsigned FULL = 0xffffffffu;
     extern __shared__ uint4 ring[];
     constexpr int LOG2G = G == 32 ? 5 : G == 16 ? 4 : G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
-    const int64_t gid = (int64_t(blockIdx.x) * kRingThreads + threadIdx.x) >> LOG2G;
+    const int64_t gid = (int64_t(blockIdx.x) * ring_threads(MODE) + threadIdx.x) >> LOG2G;
     const int64_t n_tiles_pad = (P.n_tiles + (32 / G) - 1) / (32 / G) * (32 / G);
     const int gl = threadIdx.x & (G - 1);
     const int lane = threadIdx.x & 31;
@@ -1207,9 +1210,10 @@ void launch_ring(const Params &P, cudaStream_t st) {
     // tile groups padded to whole warps, then the empty-row groups
     const int64_t per_warp = 32 / G;
     const int64_t groups = (P.n_tiles + per_warp - 1) / per_warp * per_warp + P.n_zero;
-    const unsigned grid = unsigned((groups + kRingThreads / G - 1) / (kRingThreads / G));
+    constexpr int TPB = ring_threads(MODE);
+    const unsigned grid = unsigned((groups + TPB / G - 1) / (TPB / G));
     // ring: D slots x NV vectors x 16 bytes for every lane of the block
-    const size_t smem = size_t(kRingThreads) * D * NV * 16;
+    const size_t smem = size_t(TPB) * D * NV * 16;
     // the shared-memory limit is an attribute of the function in each device's
     // context: set it once per device (a race only repeats the same call)
     static std::atomic<uint64_t> configured{0};
@@ -1221,7 +1225,7 @@ void launch_ring(const Params &P, cudaStream_t st) {
                              int(smem));
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    k_tiles_ring<T, VEC, NV, G, MODE, D><<<grid, kRingThreads, smem, st>>>(P);
+    k_tiles_ring<T, VEC, NV, G, MODE, D><<<grid, TPB, smem, st>>>(P);
 }
 
 template <typename T, int VEC, int NV, int MODE>
