@@ -36,7 +36,7 @@ def test_rmat22_shape_and_schedule(big):
     wl, g, _ = big
     assert (wl.N, wl.E, wl.H, wl.feature_dtype) == (1 << 22, 1 << 26, 128, torch.bfloat16)
     s = g.stats
-    assert s["tile_edges"] == 512 and s["tiles"] == wl.E // 512
+    assert s["tile_edges"] == 256 and s["tiles"] == wl.E // 256
     assert s["long_spanning_rows_f"] > 100 and s["max_degree_f"] > 100_000
     assert 0 < s["nonempty_rows_f"] < wl.N
 
