@@ -410,9 +410,16 @@ def our_arm(args):
 
     # lowering (once per topology; reported, not part of the step).  The first
     # call also pays the library's one-time CUDA module loading, so it is
-    # timed separately from a second, warm lowering of the same topology.
+    # timed separately from a second, warm lowering of the same topology.  The
+    # first graph is released before the second lowering, so that its
+    # workspace comes from torch's cache rather than from a new device
+    # allocation, whose time varies from run to run.
     lower_ms = []
+    g = None
     for _ in range(2):
+        if g is not None:
+            g.close()
+            g = None
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         g = agb.ag_graph_lower(wl.src, wl.dst, wl.N)
