@@ -22,6 +22,7 @@ oracle on a bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -195,31 +196,44 @@ def ncu_l2_hit(workload, kernel_op):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples of SM clock and throttle reasons during the timed
+    region: sampled every 20 ms, and only the samples whose timestamps fall
+    between the region's first launch and its end are kept (the sampler
+    starts early and stops late; its samples of the idle GPU around the
+    region would otherwise dilute the median under load)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
         self.out = tempfile.NamedTemporaryFile(prefix="clocks", suffix=".csv", delete=False)
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
             self.proc = None
         return self
 
+    def begin(self):
+        """Marks the start of the region (call right before its first launch)."""
+        self.t0 = datetime.datetime.now()
+
+    def end(self):
+        """Marks the end of the region (call after its final synchronize)."""
+        self.t1 = datetime.datetime.now()
+
     def __exit__(self, *a):
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -232,24 +246,26 @@ class ClockSampler:
             rows = [ln.split(",") for ln in open(self.out.name).read().splitlines() if ln.strip()]
         finally:
             os.unlink(self.out.name)
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        parsed = []
         for r in rows:
             r = [x.strip() for x in r]
-            if len(r) < 9:
+            if len(r) < 10:
                 continue
             try:
-                sm.append(float(r[1]))
-                smax.append(float(r[2]))
+                stamp = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f")
+                parsed.append((stamp, float(r[2]), float(r[3]), r[6:10]))
             except ValueError:
                 continue
-            for name, val in zip(names, r[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        window = "timed region"
+        inside = [p for p in parsed if self.t0 and self.t1 and self.t0 <= p[0] <= self.t1]
+        if not inside:  # a region shorter than the sampling interval
+            inside, window = parsed, "around the timed region"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": window}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = {name for p in inside for name, val in zip(names, p[3]) if val.lower().startswith("active")}
+        return {"sm_mhz": statistics.median(p[1] for p in inside), "sm_max_mhz": max(p[2] for p in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -448,6 +464,7 @@ def our_arm(args):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        clk.begin()
         start.record(stream)
         for k in range(K):
             step()
@@ -455,6 +472,7 @@ def our_arm(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        clk.end()
     clocks = clk.summary()
     ms = start.elapsed_time(end)
     ms = max_over_ranks(ms, dev)

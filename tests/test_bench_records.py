@@ -54,3 +54,32 @@ def test_source_hash_ignores_comments_and_blank_lines(edit):
     other = code.replace("// one", "// another") if edit == "comment" else code.replace("{\n", "{\n\n")
     assert bench.code_only(code) == bench.code_only(other)
     assert bench.code_only(code) != bench.code_only(code.replace("return 1", "return 2"))
+
+
+def test_clock_summary_keeps_the_samples_of_the_timed_region():
+    import datetime
+    clk = bench.ClockSampler(0)
+    base = datetime.datetime(2026, 1, 2, 3, 4, 5)
+    lines = []
+    for k, mhz in enumerate([345, 345, 1965, 1950, 1965, 345]):   # idle, idle, load x3, idle
+        stamp = (base + datetime.timedelta(milliseconds=20 * k)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        cap = "Active" if k == 3 else "Not Active"
+        lines.append(f"{stamp}, 0, {mhz}, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, {cap}")
+    clk.out.write("\n".join(lines).encode() + b"\n")
+    clk.t0 = base + datetime.timedelta(milliseconds=30)
+    clk.t1 = base + datetime.timedelta(milliseconds=90)
+    s = clk.summary()
+    assert s["samples"] == 3 and s["sm_mhz"] == 1965 and s["window"] == "timed region"
+    assert s["reasons"] == ["sw_power_cap"] and s["sm_max_mhz"] == 1965
+
+
+def test_clock_summary_falls_back_when_the_region_is_shorter_than_a_sample():
+    import datetime
+    clk = bench.ClockSampler(0)
+    base = datetime.datetime(2026, 1, 2, 3, 4, 5)
+    stamp = base.strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    clk.out.write(f"{stamp}, 0, 1900, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Not Active\n".encode())
+    clk.t0 = base + datetime.timedelta(milliseconds=5)
+    clk.t1 = base + datetime.timedelta(milliseconds=8)
+    s = clk.summary()
+    assert s["samples"] == 1 and s["window"] == "around the timed region" and s["reasons"] == []
