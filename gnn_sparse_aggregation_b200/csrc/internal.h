@@ -33,7 +33,7 @@ constexpr int kWindowShift = AG_WINDOW_SHIFT;
 // ordinal of chunk c in window b into its position in the chunk sorted by
 // window (slot + delta).  Built when the graph has at most kStageMaxWindows
 // windows.
-constexpr int kStageChunk = 4096;
+constexpr int kStageChunk = 2048;  // (R-MAT-22 step 1 % faster than with 4096; 1024 slower)
 constexpr int kStageMaxWindows = 256;
 
 constexpr size_t kAlign = 256;
